@@ -1,0 +1,108 @@
+"""Plant plausible mistakes in the oracle (CPU only) and check that the pins
+in ``test_oracle_pins`` catch every one of them."""
+
+import numpy as np
+import pytest
+
+import oracle.moe_oracle as om
+from tests import test_oracle_pins as pins
+
+
+def _route_weights_from_c(x, Wr, bias, cfg):
+    _, s, c = om.router_scores(x, Wr, bias)
+    ids, margin = om.group_limited_topk(c, cfg.n_group, cfg.topk_group, cfg.top_k)
+    return ids, om.routing_weights(c, ids, cfg.routed_scaling_factor), margin, s
+
+
+def _double_scaling(s, ids, rsf, norm=True):
+    sel = np.take_along_axis(s.astype(np.float64), ids.astype(np.int64), axis=1)
+    return rsf * rsf * sel / sel.sum(axis=1, keepdims=True)
+
+
+def _no_group_step(c, n_group, topk_group, top_k):
+    return _ORIG_GLT(c, n_group, n_group, top_k)
+
+
+def _group_score_max(c, n_group, topk_group, top_k):
+    T, E = c.shape
+    gs = E // n_group
+    G = c.reshape(T, n_group, gs).max(axis=2)
+    kept = np.argsort(-G, axis=1, kind="stable")[:, :topk_group]
+    mask = np.zeros((T, n_group), bool)
+    np.put_along_axis(mask, kept, True, axis=1)
+    cand = np.where(np.repeat(mask, gs, axis=1), c.astype(np.float64), -np.inf)
+    ids = np.argsort(-cand, axis=1, kind="stable")[:, :top_k].astype(np.int32)
+    return ids, np.full(T, np.inf)
+
+
+def _gate_up_swapped(x, w13, w2):
+    I = w13.shape[0] // 2
+    return _ORIG_SWIGLU(x, np.concatenate([w13[I:], w13[:I]]), w2)
+
+
+def _w2_transposed_use(x, w13, w2):
+    # uses w2 as if it were stored [I, H] (wrong orientation), only meaningful when square
+    I = w13.shape[0] // 2
+    xd = x.astype(np.float64)
+    h = om._silu(xd @ w13[:I].T) * (xd @ w13[I:].T)
+    return h @ (w2.reshape(w2.shape[1], w2.shape[0]).astype(np.float64))
+
+
+_ORIG_GLT = om.group_limited_topk
+_ORIG_SWIGLU = om.swiglu_mlp
+
+
+def _scaled_shared(*args, **kw):
+    out, ids, w, m = _ORIG_FWD(*args, **kw)
+    x, ws13, ws2, cfg = args[0], args[5], args[6], args[7]
+    if ws13 is not None:
+        out = out + (cfg.routed_scaling_factor - 1.0) * _ORIG_SWIGLU(x, ws13, ws2)
+    return out, ids, w, m
+
+
+_ORIG_FWD = om.moe_forward
+
+PIN_TESTS = [
+    lambda: pins.test_hand_worked_golden_example(),
+    lambda: [pins.test_selection_matches_brute_force(*a) for a in
+             [(8, 4, 2, 2), (16, 4, 2, 4), (12, 3, 2, 3)]],
+    lambda: pins.test_bias_forces_selection_but_not_weights(),
+    lambda: pins.test_weights_sum_to_scaling_factor_once(),
+    lambda: pins.test_identical_experts_give_scaled_dense_mlp(),
+    lambda: pins.test_single_expert_is_textbook_swiglu_plus_shared(),
+    lambda: pins.test_swiglu_gate_up_order_and_w2_orientation(),
+]
+
+MUTATIONS = {
+    "weights_from_bias_corrected_scores": [(pins, "route", _route_weights_from_c),
+                                           (om, "route", _route_weights_from_c)],
+    "scaling_applied_twice": [(om, "routing_weights", _double_scaling),
+                              (pins, "routing_weights", _double_scaling)],
+    "group_step_dropped": [(om, "group_limited_topk", _no_group_step),
+                           (pins, "group_limited_topk", _no_group_step)],
+    "group_score_is_max": [(om, "group_limited_topk", _group_score_max),
+                           (pins, "group_limited_topk", _group_score_max)],
+    "gate_up_swapped": [(om, "swiglu_mlp", _gate_up_swapped),
+                        (pins, "swiglu_mlp", _gate_up_swapped)],
+    "w2_misoriented": [(om, "swiglu_mlp", _w2_transposed_use),
+                       (pins, "swiglu_mlp", _w2_transposed_use)],
+    "shared_expert_scaled": [(pins, "moe_forward", _scaled_shared)],
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    for mod, attr, fn in MUTATIONS[name]:
+        monkeypatch.setattr(mod, attr, fn)
+    failures = 0
+    for pin in PIN_TESTS:
+        try:
+            pin()
+        except Exception:  # AssertionError, or a shape error from a wrong layout
+            failures += 1
+    assert failures >= 1, f"no pin caught the planted mistake {name!r}"
+
+
+def test_unmutated_oracle_passes_every_pin():
+    for pin in PIN_TESTS:
+        pin()
