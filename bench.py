@@ -1,0 +1,395 @@
+"""Benchmark of the routed MoE block forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+One step = one full block forward (router, permutation, grouped SwiGLU
+experts, shared expert and combine) over one batch of seeded synthetic
+tokens, inputs resident in HBM.  The default workload is the 19,412-token
+layer (21 latent frames x 30x30 patches + 512 text tokens, H=2048, 128
+experts, top-8).  Under torchrun every rank runs its own batch of the same
+size on its own GPU (token data parallelism: no collective on the data path;
+weak scaling); the timed region is bracketed by a barrier and a device
+synchronise on both sides and the slowest rank's time is reported.
+
+``--impl reference`` times the CPU oracle (the only reference
+implementation: the source pages ship no code) on a bounded token sample of
+the same workload, on rank 0 only.
+
+Prints one JSON line (rank 0).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from routed_moe_layer_b200 import inputs, ops  # noqa: E402
+from routed_moe_layer_b200.ops import BlockConfig  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and TFLOP/s at T~19.4k bf16; % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 9  # router, 3 permute, gather, expert up, expert down, shared up, combine
+
+
+def flops_per_token(cfg: BlockConfig) -> float:
+    """Algorithmic FLOPs of one token: router GEMM, top_k SwiGLU experts, shared expert."""
+    return (2.0 * cfg.E * cfg.H + cfg.top_k * 6.0 * cfg.H * cfg.I + 6.0 * cfg.H * cfg.I_shared)
+
+
+def algorithmic_bytes(cfg: BlockConfig, experts_used: int) -> float:
+    """Weights of the experts that receive a token + shared + router + x in + out."""
+    per_expert = 3.0 * cfg.I * cfg.H * 2
+    return (experts_used * per_expert + 3.0 * cfg.I_shared * cfg.H * 2 + cfg.E * cfg.H * 4 +
+            cfg.E * 4 + 2.0 * cfg.T * cfg.H * 2)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+
+    def stop(self):
+        if self._thr is not None:
+            self._stop.set()
+            self._thr.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"],
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def _dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_sample(cfg_id: int, target_s: float = 12.0, d_cpu=None):
+    """Times the CPU oracle on a bounded sample of the workload's tokens.
+    Returns (tokens_per_s, cores, sample description)."""
+    import oracle
+    from tests import parity
+
+    wl = inputs.WORKLOADS[cfg_id]
+    cfg = BlockConfig(T=wl.T, H=wl.H)
+    if d_cpu is None:
+        d_cpu = inputs.workload_inputs(cfg_id)
+    dn = parity.np_inputs(d_cpu)
+    ocfg = parity.oracle_cfg(cfg)
+    rng = np.random.default_rng(0)
+    n = 16
+    t_used = 0.0
+    done = 0
+    while True:
+        toks = rng.choice(wl.T, n, replace=False)
+        t0 = time.perf_counter()
+        oracle.moe_forward_tokens(toks, dn["x"], dn["Wr"], dn["bias"], dn["w13"], dn["w2"],
+                                  dn["ws13"], dn["ws2"], ocfg)
+        dt = time.perf_counter() - t0
+        t_used += dt
+        done += n
+        if t_used >= target_s or done >= wl.T:
+            break
+        n = int(min(wl.T - done, max(n, n * max(1.0, (target_s - t_used) / max(dt, 1e-3)))))
+        n = max(1, min(n, 4096))
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    return done / t_used, int(cores), (f"{done} tokens of {wl.name} drawn at random, "
+                                       f"float64 NumPy oracle, {t_used:.1f} s")
+
+
+def run_reference(args, world, rank):
+    """CPU oracle arm: bounded token sample per step, rank 0 only."""
+    if rank != 0:
+        return
+    wl = inputs.WORKLOADS[args.config]
+    cfg = BlockConfig(T=wl.T, H=wl.H)
+    import oracle
+    from tests import parity
+    d_cpu = inputs.workload_inputs(args.config)
+    dn = parity.np_inputs(d_cpu)
+    ocfg = parity.oracle_cfg(cfg)
+    per_step = max(1, min(wl.T, args.ref_tokens))
+    rng = np.random.default_rng(1)
+    for _ in range(args.warmup if args.ref_warmup else 0):
+        toks = rng.choice(wl.T, per_step, replace=False)
+        oracle.moe_forward_tokens(toks, dn["x"], dn["Wr"], dn["bias"], dn["w13"], dn["w2"],
+                                  dn["ws13"], dn["ws2"], ocfg)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        toks = rng.choice(wl.T, per_step, replace=False)
+        oracle.moe_forward_tokens(toks, dn["x"], dn["Wr"], dn["bias"], dn["w13"], dn["w2"],
+                                  dn["ws13"], dn["ws2"], ocfg)
+    dt = time.perf_counter() - t0
+    tps = per_step * args.steps / dt
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": 128, "I": 768,
+                   "top_k": 8, "tokens_per_step_sampled": per_step},
+        "tflops": tps * flops_per_token(cfg) / 1e12,
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
+                         "sample": f"{per_step} random tokens of {wl.name} per step"},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    wl = inputs.WORKLOADS[args.config]
+    cfg = BlockConfig(T=wl.T, H=wl.H)
+    layers = wl.layers
+    # weights: identical on every rank; tokens: a different batch per rank
+    gen_dev = dev if layers > 1 else "cpu"
+    weights = []
+    for l in range(layers):
+        wd = inputs.make_weights(wl.H, wl.seed, device=gen_dev, layer=l,
+                                 hot_experts=wl.hot_experts, hot_bias=wl.hot_bias)
+        weights.append({k: (None if v is None else v.to(dev)) for k, v in wd.items()})
+    x_host = inputs.make_tokens(wl.T, wl.H, wl.seed + 1000 * rank).pin_memory()
+    x = x_host.to(dev)
+    ws = ops.alloc_workspace(ops.workspace_bytes(cfg), dev)
+    out = torch.empty_like(x)
+    xn_buf = torch.empty_like(x)
+    ids = torch.empty((wl.T, cfg.top_k), dtype=torch.int32, device=dev)
+
+    def step(xin, timer=None):
+        if layers == 1:
+            w = weights[0]
+            return ops.forward(xin, w["Wr"], w["bias"], w["w13"], w["w2"], w["ws13"], w["ws2"],
+                               cfg, out=out, workspace=ws, timer=timer, topk_ids=ids)
+        # residual stack: x <- x + block_l(RMSNorm(x)), updated in place in `out`
+        out.copy_(xin)
+        for l, w in enumerate(weights):
+            ops.rmsnorm(out, eps=1e-6, out=xn_buf)
+            ops.forward(xn_buf, w["Wr"], w["bias"], w["w13"], w["w2"], w["ws13"], w["ws2"], cfg,
+                        residual=out, out=out, workspace=ws, timer=timer if l == 0 else None,
+                        topk_ids=ids)
+        return out
+
+    for _ in range(args.warmup):
+        step(x)
+    torch.cuda.synchronize()
+    code, site = ops.read_device_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {ops.status_string(code)} at {site}")
+
+    stream = torch.cuda.current_stream()
+    timers = [ops.StageTimer() for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(x, timer=timers[i])
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    sampler.stop()
+    _barrier(world)
+    ms_local = ev0.elapsed_time(ev1) / args.steps
+    ms = _max_over_ranks(ms_local, world)
+    code, site = ops.read_device_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {ops.status_string(code)} at {site}")
+
+    # per-stage device times (stage 'expert_up' is exactly one kernel launch)
+    per_stage = {k: float(np.mean([t.stage_ms()[k] for t in timers])) for k in ops.STAGES}
+    counts = torch.bincount(ids.reshape(-1).long(), minlength=cfg.E)
+    experts_used = int((counts > 0).sum().item())
+
+    # end to end: pinned host tokens -> device -> block -> host, every step
+    out_host = torch.empty_like(x_host).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        y = step(x_dev)
+        out_host.copy_(y, non_blocking=True)
+    _barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        y = step(x_dev)
+        out_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        tok_per_step = wl.T * layers
+        total_tokens = tok_per_step * world
+        value = total_tokens / (ms * 1e-3)
+        fpt = flops_per_token(cfg)
+        tflops = value * fpt / 1e12
+        R = wl.T * cfg.top_k
+        up_flops = 2.0 * R * cfg.H * (2 * cfg.I)
+        up_ms = per_stage["expert_up"]
+        peak_tf = peaks["bf16_tflops"]
+        achieved = up_flops / (up_ms * 1e-3) / 1e12
+        layer_ms = ms / layers
+        hbm_bytes = algorithmic_bytes(cfg, experts_used)
+        rf = {"bound": "tensor", "kernel": "grouped_gemm_kernel<SwiGLU> (expert up)",
+              "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+              "frac": achieved / peak_tf,
+              "peak_source": f"{peak_src} bf16 dense burst",
+              "traffic": None,
+              "layer_roofline_frac": max(fpt * wl.T / peak_tf / 1e12,
+                                         hbm_bytes / peaks["hbm_gbs"] / 1e9) / (layer_ms * 1e-3)}
+        cpu_tps, cores, sample = (None, None, None)
+        if world == 1 and not args.no_cpu_baseline:
+            cpu_tps, cores, sample = cpu_oracle_sample(args.config, target_s=args.cpu_seconds)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded normal/uniform tensors of the workload's shapes)",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": cfg.E, "I": cfg.I,
+                       "I_shared": cfg.I_shared, "top_k": cfg.top_k, "n_group": cfg.n_group,
+                       "topk_group": cfg.topk_group, "layers": layers,
+                       "tokens_per_gpu_per_step": tok_per_step,
+                       "l2": "inputs larger than L2: 1.2 GB of expert weights read per layer"},
+            "tflops": tflops,
+            "roofline": rf,
+            "stage_ms": per_stage,
+            "experts_used": experts_used,
+            "cpu_baseline": None if cpu_tps is None else {
+                "value": cpu_tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                "sample": sample},
+            "e2e": {"value": total_tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(x_host.numel() * 2),
+                    "d2h_bytes_per_step": int(out_host.numel() * 2)},
+            "gpu_launches": (KERNELS_PER_STEP + (1 if layers > 1 else 0)) * layers * args.steps,
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2, choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-tokens", type=int, default=64,
+                    help="tokens per step for --impl reference (bounded CPU sample)")
+    ap.add_argument("--ref-warmup", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        raise SystemExit("--warmup must be >= 3")
+    world, rank, local = _dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,187 @@
+/*
+ * routed_moe.h -- C ABI of libroutedmoe.so: forward pass of a DeepSeek-V3-style
+ * routed Mixture-of-Experts block (the LingBot-Video MoE DiT block) on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the block computes (sources are web pages, cited by title + section):
+ *   [S1] prhub report "sglang PR #32341: LingBot-Video MoE 30B", section
+ *        "实现拆解" (implementation breakdown) step 1 and section "关键源码片段"
+ *        (key source snippets), LingBotVideoSparseMoeBlock / LingBotVideoRouter.
+ *   [S2] xxqk.cn article "vLLM-Omni 原生推理 LingBot-Video", section
+ *        "MoE 实现的源码级要点" (source-level MoE notes).
+ *
+ *   router  : logits = x . Wr^T (fp32), s = sigmoid(logits), c = s + bias;
+ *             group score = sum of the top-2 c of each of n_group groups;
+ *             keep the topk_group best groups; ids = top_k largest c among
+ *             their experts; w = routed_scaling_factor * s[ids] / sum s[ids]
+ *             (raw scores, renormalised, scaled once)            [S1] step 1, [S2]
+ *   experts : y_e(x) = (silu(x . W13[e,0:I]^T) * (x . W13[e,I:2I]^T)) . W2[e]^T
+ *             with w13 packed [E, 2I, H] gate rows then up rows   [S1] snippets
+ *   output  : out = sum_i w_i * y_{ids_i}(x) + shared(x) [+ residual]
+ *             (fp32 weighted restore; shared expert added unscaled) [S1], [S2]
+ *
+ * Conventions for every entry point
+ *   - Linear layers are y = x . W^T with W row-major [out, in].
+ *   - Pointers named "device" are CUDA device memory owned by the caller;
+ *     the library never allocates, frees or keeps them.  Host pointers are
+ *     only read during the call.
+ *   - "stream" is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it and never synchronise the host, except
+ *     moe_read_device_status.
+ *   - bf16 tensors are IEEE bfloat16, row-major and contiguous.
+ *   - Every call checks its arguments first and launches nothing when it
+ *     returns an error.  T == 0 is valid and does nothing.
+ *   - Calls that share a workspace must not overlap on the device.
+ */
+#ifndef ROUTED_MOE_H
+#define ROUTED_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,        /* null pointer, negative size, inconsistent cfg */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,  /* shape outside what the kernels implement */
+  MOE_ERR_WORKSPACE = 3,          /* workspace missing, misaligned or too small */
+  MOE_ERR_CUDA = 4,               /* a CUDA runtime / driver call failed */
+  MOE_ERR_DEVICE_TIMEOUT = 5,     /* a device-side wait ran past its limit */
+  MOE_ERR_DEVICE_INDEX = 6,       /* a kernel met an expert id outside [0, E) */
+  MOE_ERR_NO_DEVICE = 7           /* no sm_100 device current */
+} moe_status_t;
+
+/* Block configuration.  Defaults of the LingBot-Video MoE model ([S1]
+ * "实现拆解" step 3): E=128, I=768, top_k=8, n_group=4, topk_group=2,
+ * routed_scaling_factor=2.5, norm_topk_prob=1, one shared expert of I_shared=768. */
+typedef struct {
+  int32_t T;                      /* tokens (rows of x) */
+  int32_t H;                      /* hidden size; multiple of 64 */
+  int32_t E;                      /* routed experts; 1..128, divisible by n_group */
+  int32_t I;                      /* moe_intermediate_size; multiple of 64 */
+  int32_t I_shared;               /* shared expert intermediate size; 0 = none, else multiple of 64 */
+  int32_t top_k;                  /* experts per token; 1..16 */
+  int32_t n_group;                /* expert groups */
+  int32_t topk_group;             /* groups kept per token */
+  float routed_scaling_factor;    /* applied once, inside the router */
+  int32_t norm_topk_prob;         /* 1: renormalise the chosen scores to sum 1 first */
+  int32_t flags;                  /* reserved, must be 0 */
+} moe_cfg_t;
+
+/* Stages of moe_forward, in launch order (for stage_events). */
+#define MOE_STAGE_ROUTER 0
+#define MOE_STAGE_PERMUTE 1
+#define MOE_STAGE_EXPERT_UP 2
+#define MOE_STAGE_EXPERT_DOWN 3
+#define MOE_STAGE_SHARED_UP 4
+#define MOE_STAGE_COMBINE 5
+#define MOE_NUM_STAGES 6
+
+/* Optional arguments of moe_forward (pass NULL for all defaults). */
+typedef struct {
+  const void* residual;   /* device bf16 [T,H] or NULL: out = residual + block(x);
+                             may be the same buffer as out */
+  int32_t* topk_ids;      /* device int32 [T,top_k] or NULL: also write the routing ids */
+  float* topk_w;          /* device fp32 [T,top_k] or NULL: also write the routing weights */
+  void** stage_events;    /* host array of MOE_NUM_STAGES+1 cudaEvent_t or NULL: event i is
+                             recorded on stream before stage i, the last one after the last */
+  int64_t wait_timeout_ns;/* limit of every device-side wait; 0 = 2 s */
+} moe_forward_opts_t;
+
+/* Human-readable name of a status code; never NULL. */
+MOE_API const char* moe_status_string(int32_t status);
+
+/* Checks cfg against the limits above; MOE_OK or the first violation.
+ * [S1] "风险与影响" item 4 names the divisibility of E by n_group and a
+ * group of at least 2 experts (the per-group top-2) as assumptions. */
+MOE_API int32_t moe_check_config(const moe_cfg_t* cfg);
+
+/* Workspace bytes needed by moe_route / moe_permute / moe_forward for cfg
+ * (0 when cfg is invalid).  The workspace is device memory, 256-byte aligned. */
+MOE_API size_t moe_route_workspace_bytes(const moe_cfg_t* cfg);
+MOE_API size_t moe_permute_workspace_bytes(const moe_cfg_t* cfg);
+MOE_API size_t moe_workspace_bytes(const moe_cfg_t* cfg);
+
+/* Router ([S1] step 1, LingBotVideoRouter.forward(tokens) -> (top_indices,
+ * top_scores); [S2] asymmetric routing).
+ *   x        device bf16 [T,H]
+ *   Wr       device fp32 [E,H]   router weight (kept in fp32)
+ *   bias     device fp32 [E]     e_score_correction_bias (selection only)
+ *   topk_ids device int32 [T,top_k] out: expert ids, descending c, ties to the lower id
+ *   topk_w   device fp32 [T,top_k] out: gating weights, same order
+ *   workspace may be NULL when moe_route_workspace_bytes(cfg) == 0. */
+MOE_API int32_t moe_route(const void* x, const float* Wr, const float* bias, const moe_cfg_t* cfg,
+                  int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/* Token -> expert permutation ([S2] "_reorder_tokens": tokens regrouped per
+ * expert before the grouped GEMMs).  Rows are ordered by expert, then by
+ * token, so the permutation is unique and deterministic.
+ *   topk_ids       device int32 [T,top_k], every id in [0,E)
+ *   topk_w         device fp32 [T,top_k] or NULL
+ *   x              device bf16 [T,H] or NULL (then xp is not written)
+ *   expert_offsets device int32 [E+1] out: first row of each expert, [E] = T*top_k
+ *   row_of         device int32 [T*top_k] out: row of (token t, slot j) at t*top_k+j
+ *   tok_of         device int32 [T*top_k] out: token of each row
+ *   w_of           device fp32 [T*top_k] out or NULL: weight of each row
+ *   xp             device bf16 [T*top_k, H] out or NULL: xp[row] = x[tok_of[row]]
+ * An id outside [0,E) is skipped and leaves MOE_ERR_DEVICE_INDEX in the
+ * workspace status word (see moe_read_device_status). */
+MOE_API int32_t moe_permute(const int32_t* topk_ids, const float* topk_w, const void* x,
+                    const moe_cfg_t* cfg, int32_t* expert_offsets, int32_t* row_of,
+                    int32_t* tok_of, float* w_of, void* xp, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* Whole block forward ([S1] LingBotVideoSparseMoeBlock.forward: router ->
+ * grouped SwiGLU experts with the router weight applied on the output ->
+ * fp32 restore ([S2] "_restore_tokens") -> + shared expert, unscaled).
+ *   x     device bf16 [T,H]          block input
+ *   Wr    device fp32 [E,H], bias device fp32 [E]
+ *   w13   device bf16 [E,2I,H]       gate rows 0..I-1, up rows I..2I-1 (non-interleaved)
+ *   w2    device bf16 [E,H,I]
+ *   ws13  device bf16 [2I_s,H], ws2 device bf16 [H,I_s]  (NULL when I_shared == 0)
+ *   out   device bf16 [T,H]          must not overlap x
+ *   opts  host pointer or NULL
+ * The result is rounded to bf16 once, after an fp32 sum in a fixed order
+ * (slots 0..top_k-1, then the shared expert, then the residual), so it is
+ * bitwise reproducible and each token's output does not depend on the
+ * other tokens of the call. */
+MOE_API int32_t moe_forward(const void* x, const float* Wr, const float* bias, const void* w13,
+                    const void* w2, const void* ws13, const void* ws2, const moe_cfg_t* cfg,
+                    void* out, const moe_forward_opts_t* opts, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* RMSNorm with fp32 accumulation ([S2]: RMSNorm accumulates in fp32), for a
+ * residual stack of blocks: xn = bf16(x * rsqrt(mean(x^2) + eps) * gamma).
+ *   x device bf16 [T,H]; gamma device fp32 [H] or NULL (= 1); xn device bf16 [T,H]. */
+MOE_API int32_t moe_rmsnorm(const void* x, const float* gamma, float eps, int32_t T, int32_t H,
+                    void* xn, void* stream);
+
+/* Waits for stream, then reads and clears the device status word that the
+ * kernels of moe_forward / moe_permute leave in workspace (MOE_OK, or the
+ * first device-side error of the last call).  *site receives where the
+ * error arose (kernel-specific; may be NULL). */
+MOE_API int32_t moe_read_device_status(void* workspace, int32_t* site, void* stream);
+
+/* Failure-detection self test: launches one kernel whose thread waits on a
+ * device flag that nothing sets, with the same bounded wait that every
+ * pipeline wait of the library uses.  The wait gives up after timeout_ns and
+ * leaves MOE_ERR_DEVICE_TIMEOUT in the status word of workspace (>= 256 bytes);
+ * the context stays usable. */
+MOE_API int32_t moe_selftest_wait_timeout(void* workspace, int64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROUTED_MOE_H */

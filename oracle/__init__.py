@@ -22,5 +22,6 @@ from .moe_oracle import (  # noqa: F401
     swiglu_mlp,
     moe_forward,
     moe_forward_tokens,
+    permutation,
     rmsnorm,
 )

@@ -170,6 +170,29 @@ def route(x, Wr, bias, cfg: MoeConfig):
 
 
 # ----------------------------------------------------------------------------
+# Token reorder ([S2] "_reorder_tokens": rows regrouped by expert before the
+# grouped expert GEMMs).  Reading: rows ordered by expert, then token, which
+# makes the permutation unique.
+# ----------------------------------------------------------------------------
+def permutation(ids: np.ndarray, E: int):
+    """Returns (expert_offsets [E+1], row_of [T*k], tok_of [T*k]), int64.
+
+    The (token, slot) entries flattened as t*k + j are sorted by expert with a
+    stable sort (a token holds each expert at most once, so equal experts keep
+    token order); row_of maps an entry to its row, tok_of a row to its token.
+    """
+    T, k = ids.shape
+    flat = ids.reshape(-1).astype(np.int64)
+    order = np.argsort(flat, kind="stable")          # row -> flattened entry
+    row_of = np.empty(T * k, dtype=np.int64)
+    row_of[order] = np.arange(T * k)
+    tok_of = order // k
+    counts = np.bincount(flat, minlength=E)
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    return offsets, row_of, tok_of
+
+
+# ----------------------------------------------------------------------------
 # Experts ([S1] "关键源码片段": activation silu, gated, non-interleaved w13)
 # ----------------------------------------------------------------------------
 def _silu(a: np.ndarray) -> np.ndarray:

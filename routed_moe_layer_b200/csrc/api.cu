@@ -1,0 +1,372 @@
+// C ABI of libroutedmoe.so (declared in include/routed_moe.h): argument
+// checks, workspace layout, tensor-map set-up and the launch sequence of the
+// block forward (sglang PR #32341 report, LingBotVideoSparseMoeBlock.forward:
+// router -> grouped SwiGLU experts weighted on the output -> fp32 restore ->
+// + unscaled shared expert).
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "routed_moe.h"
+
+using namespace rmoe;
+
+namespace {
+
+constexpr size_t WS_ALIGN = 256;
+constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s
+constexpr int MAX_E = 128;
+constexpr int MAX_TOPK = 16;
+constexpr int MAX_NGROUP = 32;
+constexpr int MAX_DIM = 16384;
+
+size_t align_up(size_t v) { return (v + WS_ALIGN - 1) & ~(WS_ALIGN - 1); }
+
+int32_t check_cfg(const moe_cfg_t* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->H <= 0 || c->E <= 0 || c->I <= 0 || c->I_shared < 0 || c->top_k <= 0 ||
+      c->n_group <= 0 || c->topk_group <= 0 || c->flags != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
+  if (c->norm_topk_prob != 0 && c->norm_topk_prob != 1) return MOE_ERR_INVALID_ARG;
+  // the group-limited top-k assumes E divisible by n_group and, when groups
+  // are actually dropped, at least two experts per group (the per-group top-2)
+  if (c->E % c->n_group != 0) return MOE_ERR_INVALID_ARG;
+  if (c->topk_group > c->n_group) return MOE_ERR_INVALID_ARG;
+  const int gs = c->E / c->n_group;
+  if (c->topk_group < c->n_group && gs < 2) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)c->topk_group * gs < c->top_k) return MOE_ERR_INVALID_ARG;
+  if (c->E > MAX_E || c->top_k > MAX_TOPK || c->n_group > MAX_NGROUP)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (c->H % 64 != 0 || c->I % 64 != 0 || c->I_shared % 64 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (c->H > MAX_DIM || c->I > MAX_DIM || c->I_shared > MAX_DIM) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((int64_t)c->T * c->top_k > (int64_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+struct FwdLayout {
+  size_t status, ids, w, blk_hist, offsets, mtiles, row_of, tok_of, w_of, xp, h, hs, total;
+};
+
+FwdLayout fwd_layout(const moe_cfg_t& c) {
+  FwdLayout L;
+  const size_t T = c.T, R = T * c.top_k, E = c.E;
+  const size_t nblk = (T + PERMUTE_TOK - 1) / PERMUTE_TOK;
+  size_t off = 0;
+  L.status = off;   off += align_up(sizeof(DevStatus));
+  L.ids = off;      off += align_up(R * 4);
+  L.w = off;        off += align_up(R * 4);
+  L.blk_hist = off; off += align_up(nblk * E * 4);
+  L.offsets = off;  off += align_up((E + 1) * 4);
+  L.mtiles = off;   off += align_up((E + 1) * 4);
+  L.row_of = off;   off += align_up(R * 4);
+  L.tok_of = off;   off += align_up(R * 4);
+  L.w_of = off;     off += align_up(R * 4);
+  L.xp = off;       off += align_up(R * c.H * 2);  // gathered rows; reused for weighted outputs
+  L.h = off;        off += align_up(R * c.I * 2);
+  L.hs = off;       off += align_up(T * c.I_shared * 2);
+  L.total = off;
+  return L;
+}
+
+struct PermLayout {
+  size_t status, blk_hist, mtiles, total;
+};
+
+PermLayout perm_layout(const moe_cfg_t& c) {
+  PermLayout L;
+  const size_t nblk = ((size_t)c.T + PERMUTE_TOK - 1) / PERMUTE_TOK;
+  size_t off = 0;
+  L.status = off;   off += align_up(sizeof(DevStatus));
+  L.blk_hist = off; off += align_up(nblk * c.E * 4);
+  L.mtiles = off;   off += align_up((c.E + 1) * 4);
+  L.total = off;
+  return L;
+}
+
+bool ws_ok(const void* ws, size_t have, size_t need) {
+  if (need == 0) return true;
+  if (!ws || have < need) return false;
+  return (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN) == 0;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+RouterParams router_params(const moe_cfg_t& c) {
+  RouterParams p;
+  p.T = c.T;
+  p.H = c.H;
+  p.E = c.E;
+  p.top_k = c.top_k;
+  p.n_group = c.n_group;
+  p.topk_group = c.topk_group;
+  p.norm_topk_prob = c.norm_topk_prob;
+  p.rsf = c.routed_scaling_factor;
+  return p;
+}
+
+#define RMOE_TRY(expr)                       \
+  do {                                       \
+    const cudaError_t e_ = (expr);           \
+    if (e_ != cudaSuccess) return MOE_ERR_CUDA; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int32_t status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument or configuration";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE: shape outside the kernels' limits";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call failed";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT: a device-side wait ran out";
+    case MOE_ERR_DEVICE_INDEX: return "MOE_ERR_DEVICE_INDEX: an expert id outside [0, E)";
+    case MOE_ERR_NO_DEVICE: return "MOE_ERR_NO_DEVICE: no usable CUDA device";
+    default: return "unknown moe_status_t";
+  }
+}
+
+int32_t moe_check_config(const moe_cfg_t* cfg) { return check_cfg(cfg); }
+
+size_t moe_route_workspace_bytes(const moe_cfg_t* cfg) {
+  (void)cfg;
+  return 0;
+}
+
+size_t moe_permute_workspace_bytes(const moe_cfg_t* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return perm_layout(*cfg).total;
+}
+
+size_t moe_workspace_bytes(const moe_cfg_t* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return fwd_layout(*cfg).total;
+}
+
+int32_t moe_route(const void* x, const float* Wr, const float* bias, const moe_cfg_t* cfg,
+                  int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  const int32_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  (void)workspace;
+  (void)workspace_bytes;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !Wr || !bias || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_router(x, Wr, bias, router_params(*cfg), topk_ids, topk_w,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+int32_t moe_permute(const int32_t* topk_ids, const float* topk_w, const void* x,
+                    const moe_cfg_t* cfg, int32_t* expert_offsets, int32_t* row_of,
+                    int32_t* tok_of, float* w_of, void* xp, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  const int32_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!topk_ids || !expert_offsets || !row_of || !tok_of) return MOE_ERR_INVALID_ARG;
+  if (xp && !x) return MOE_ERR_INVALID_ARG;
+  const PermLayout L = perm_layout(*cfg);
+  if (!ws_ok(workspace, workspace_bytes, L.total)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = at<int>(workspace, L.status);
+  RMOE_TRY(launch_status_reset(status, s));
+  PermuteOut o;
+  o.status = status;
+  o.blk_hist = at<int>(workspace, L.blk_hist);
+  o.expert_offsets = expert_offsets;
+  o.mtile_start = at<int>(workspace, L.mtiles);
+  o.row_of = row_of;
+  o.tok_of = tok_of;
+  o.w_of = w_of;
+  o.xp = xp;
+  return cuda_status(launch_permute(topk_ids, topk_w, x, cfg->T, cfg->H, cfg->E, cfg->top_k, o, s));
+}
+
+int32_t moe_forward(const void* x, const float* Wr, const float* bias, const void* w13,
+                    const void* w2, const void* ws13, const void* ws2, const moe_cfg_t* cfg,
+                    void* out, const moe_forward_opts_t* opts, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  const int32_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  const moe_cfg_t& c = *cfg;
+  if (c.T == 0) return MOE_OK;
+  if (!x || !Wr || !bias || !w13 || !w2 || !out) return MOE_ERR_INVALID_ARG;
+  if ((c.I_shared > 0) != (ws13 != nullptr && ws2 != nullptr)) return MOE_ERR_INVALID_ARG;
+  if (out == x) return MOE_ERR_INVALID_ARG;
+  const FwdLayout L = fwd_layout(c);
+  if (!ws_ok(workspace, workspace_bytes, L.total)) return MOE_ERR_WORKSPACE;
+  if (opts && opts->wait_timeout_ns < 0) return MOE_ERR_INVALID_ARG;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void** ev = opts ? opts->stage_events : nullptr;
+  const unsigned long long timeout =
+      (opts && opts->wait_timeout_ns > 0) ? (unsigned long long)opts->wait_timeout_ns
+                                          : DEFAULT_TIMEOUT_NS;
+  const size_t T = c.T, R = T * c.top_k;
+  int* status = at<int>(workspace, L.status);
+  int32_t* ids = (opts && opts->topk_ids) ? opts->topk_ids : at<int32_t>(workspace, L.ids);
+  float* tw = (opts && opts->topk_w) ? opts->topk_w : at<float>(workspace, L.w);
+  int* offsets = at<int>(workspace, L.offsets);
+  int* mtiles = at<int>(workspace, L.mtiles);
+  int* row_of = at<int>(workspace, L.row_of);
+  __nv_bfloat16* xp = at<__nv_bfloat16>(workspace, L.xp);
+  __nv_bfloat16* h = at<__nv_bfloat16>(workspace, L.h);
+  __nv_bfloat16* hs = at<__nv_bfloat16>(workspace, L.hs);
+
+  // tensor maps (host-side descriptors, passed by value to the kernels)
+  CUtensorMap tm_xp, tm_w13, tm_h, tm_w2, tm_x, tm_ws13, tm_hs, tm_ws2;
+  RMOE_TRY(make_tmap_2d(&tm_xp, xp, R, c.H));
+  RMOE_TRY(make_tmap_3d(&tm_w13, w13, c.E, 2 * (uint64_t)c.I, c.H));
+  RMOE_TRY(make_tmap_2d(&tm_h, h, R, c.I));
+  RMOE_TRY(make_tmap_3d(&tm_w2, w2, c.E, c.H, c.I));
+  if (c.I_shared > 0) {
+    RMOE_TRY(make_tmap_2d(&tm_x, x, T, c.H));
+    RMOE_TRY(make_tmap_3d(&tm_ws13, ws13, 1, 2 * (uint64_t)c.I_shared, c.H));
+    RMOE_TRY(make_tmap_2d(&tm_hs, hs, T, c.I_shared));
+    RMOE_TRY(make_tmap_3d(&tm_ws2, ws2, 1, c.H, c.I_shared));
+  }
+  const int sms = num_sms();
+
+  auto record = [&](int i) -> cudaError_t {
+    return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
+  };
+
+  RMOE_TRY(record(MOE_STAGE_ROUTER));
+  RMOE_TRY(launch_status_reset(status, s));
+  RMOE_TRY(launch_router(x, Wr, bias, router_params(c), ids, tw, s));
+
+  RMOE_TRY(record(MOE_STAGE_PERMUTE));
+  PermuteOut o;
+  o.status = status;
+  o.blk_hist = at<int>(workspace, L.blk_hist);
+  o.expert_offsets = offsets;
+  o.mtile_start = mtiles;
+  o.row_of = row_of;
+  o.tok_of = at<int>(workspace, L.tok_of);
+  o.w_of = at<float>(workspace, L.w_of);
+  o.xp = xp;
+  RMOE_TRY(launch_permute(ids, tw, x, c.T, c.H, c.E, c.top_k, o, s));
+
+  const int mt_bound = (int)(R / MTILE) + c.E;  // every expert adds at most one partial tile
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.status = status;
+  a.timeout_ns = timeout;
+
+  RMOE_TRY(record(MOE_STAGE_EXPERT_UP));
+  {  // h = silu(xp . W13g^T) * (xp . W13u^T), per expert
+    GemmArgs g = a;
+    g.mtile_start = mtiles;
+    g.row_start = offsets;
+    g.num_groups = c.E;
+    g.n_tiles = (c.I + 127) / 128;
+    g.k_steps = c.H / 64;
+    g.n_out_tile = 128;
+    g.b_second = c.I;
+    g.out = h;
+    g.ldo = c.I;
+    g.n_valid = c.I;
+    const int grid = (int)std::min<long long>(sms, (long long)mt_bound * g.n_tiles);
+    RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_xp, tm_w13, g, grid, s));
+  }
+  RMOE_TRY(record(MOE_STAGE_EXPERT_DOWN));
+  {  // Y = w_row * (h . W2^T), per expert, written over the gathered rows
+    GemmArgs g = a;
+    g.mtile_start = mtiles;
+    g.row_start = offsets;
+    g.num_groups = c.E;
+    g.n_tiles = (c.H + 255) / 256;
+    g.k_steps = c.I / 64;
+    g.n_out_tile = 256;
+    g.b_second = 128;
+    g.out = xp;
+    g.ldo = c.H;
+    g.n_valid = c.H;
+    g.row_scale = o.w_of;
+    const int grid = (int)std::min<long long>(sms, (long long)mt_bound * g.n_tiles);
+    RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, g, grid, s));
+  }
+  RMOE_TRY(record(MOE_STAGE_SHARED_UP));
+  const void* residual = opts ? opts->residual : nullptr;
+  if (c.I_shared > 0) {
+    GemmArgs g = a;
+    g.single_rows = c.T;
+    g.n_tiles = (c.I_shared + 127) / 128;
+    g.k_steps = c.H / 64;
+    g.n_out_tile = 128;
+    g.b_second = c.I_shared;
+    g.out = hs;
+    g.ldo = c.I_shared;
+    g.n_valid = c.I_shared;
+    const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
+    RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_x, tm_ws13, g, std::min(sms, tiles), s));
+  }
+  RMOE_TRY(record(MOE_STAGE_COMBINE));
+  if (c.I_shared > 0) {
+    // out = bf16( sum_j Y[row_of[t,j]] + hs . Ws2^T [+ residual] )
+    GemmArgs g = a;
+    g.single_rows = c.T;
+    g.n_tiles = (c.H + 255) / 256;
+    g.k_steps = c.I_shared / 64;
+    g.n_out_tile = 256;
+    g.b_second = 128;
+    g.out = static_cast<__nv_bfloat16*>(out);
+    g.ldo = c.H;
+    g.n_valid = c.H;
+    g.Y = xp;
+    g.row_of = row_of;
+    g.top_k = c.top_k;
+    g.ldy = c.H;
+    g.residual = static_cast<const __nv_bfloat16*>(residual);
+    const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
+    RMOE_TRY(launch_grouped_gemm(EPI_COMBINE, tm_hs, tm_ws2, g, std::min(sms, tiles), s));
+  } else {
+    RMOE_TRY(launch_combine_rows(xp, row_of, c.T, c.H, c.top_k,
+                                 static_cast<const __nv_bfloat16*>(residual),
+                                 static_cast<__nv_bfloat16*>(out), s));
+  }
+  RMOE_TRY(record(MOE_NUM_STAGES));
+  return MOE_OK;
+}
+
+int32_t moe_rmsnorm(const void* x, const float* gamma, float eps, int32_t T, int32_t H, void* xn,
+                    void* stream) {
+  if (T < 0 || H <= 0 || H % 64 != 0 || H > MAX_DIM || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !xn) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_rmsnorm(x, gamma, eps, T, H, xn, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t moe_read_device_status(void* workspace, int32_t* site, void* stream) {
+  if (!workspace) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DevStatus h{0, 0};
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaMemset(workspace, 0, sizeof(h)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (site) *site = h.site;
+  return h.code;
+}
+
+int32_t moe_selftest_wait_timeout(void* workspace, int64_t timeout_ns, void* stream) {
+  if (!workspace || timeout_ns <= 0) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) % WS_ALIGN) != 0) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(workspace);
+  RMOE_TRY(launch_status_reset(status, s));
+  return cuda_status(launch_selftest_wait(status, (unsigned long long)timeout_ns, s));
+}
+
+}  // extern "C"

@@ -1,0 +1,82 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rmoe {
+
+struct RouterParams {
+  int T, H, E, top_k, n_group, topk_group, norm_topk_prob;
+  float rsf;
+};
+
+cudaError_t launch_router(const void* x, const float* Wr, const float* bias, const RouterParams& p,
+                          int32_t* topk_ids, float* topk_w, cudaStream_t stream);
+
+// ------------------------------------------------------------------ permute
+constexpr int PERMUTE_TOK = 256;  // tokens per counting block
+constexpr int MTILE = 128;        // rows per GEMM tile (the M of one UMMA)
+
+struct PermuteOut {
+  int* status;          // DevStatus
+  int* blk_hist;        // [nblk, E] scratch
+  int* expert_offsets;  // [E+1]
+  int* mtile_start;     // [E+1] prefix of ceil(count/MTILE), may be null
+  int* row_of;          // [T*k]
+  int* tok_of;          // [T*k]
+  float* w_of;          // [T*k] or null
+  void* xp;             // [T*k, H] bf16 or null
+};
+
+cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const void* x, int T,
+                           int H, int E, int top_k, const PermuteOut& o, cudaStream_t stream);
+
+// ------------------------------------------------------------------ grouped GEMM
+enum EpiKind { EPI_SWIGLU = 0, EPI_ROWSCALE = 1, EPI_COMBINE = 2 };
+
+struct GemmArgs {
+  // schedule: groups (experts) of rows, each cut into MTILE-row tiles
+  const int* mtile_start;  // [num_groups+1] device prefix of tiles per group; null: one group
+  const int* row_start;    // [num_groups+1] device first row of each group
+  int num_groups;
+  int single_rows;         // rows of the only group when mtile_start == null
+  int n_tiles;             // output tiles along N
+  int k_steps;             // K / 64
+  int n_out_tile;          // output columns per tile: 128 (SwiGLU) or 256
+  int b_second;            // row offset of the second 128-row half of the B tile
+  // epilogue
+  __nv_bfloat16* out;      // [rows, ldo]
+  int ldo;
+  int n_valid;             // valid output columns (N tail mask)
+  const float* row_scale;  // EPI_ROWSCALE: weight of each row
+  const __nv_bfloat16* Y;  // EPI_COMBINE: weighted expert outputs [T*k, ldy]
+  const int* row_of;       // EPI_COMBINE: [T*k]
+  int top_k;
+  int ldy;
+  const __nv_bfloat16* residual;  // EPI_COMBINE: [T, ldo] or null
+  int* status;
+  unsigned long long timeout_ns;
+};
+
+// A: 2D map over [rows, K] bf16, box 64 x 128, 128B swizzle.
+// B: 3D map over [groups, N_rows, K] bf16, box 64 x 128 x 1, 128B swizzle.
+cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K);
+cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, uint64_t groups, uint64_t n_rows,
+                         uint64_t K);
+
+cudaError_t launch_grouped_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                const GemmArgs& args, int grid, cudaStream_t stream);
+
+int num_sms();
+
+// ------------------------------------------------------------------ misc
+cudaError_t launch_rmsnorm(const void* x, const float* gamma, float eps, int T, int H, void* xn,
+                           cudaStream_t stream);
+cudaError_t launch_combine_rows(const void* Y, const int* row_of, int T, int H, int top_k,
+                                const void* residual, void* out, cudaStream_t stream);
+cudaError_t launch_status_reset(int* status, cudaStream_t stream);
+cudaError_t launch_selftest_wait(int* status, unsigned long long timeout_ns, cudaStream_t stream);
+
+}  // namespace rmoe

@@ -1,0 +1,212 @@
+// Token -> expert permutation (xxqk.cn vLLM-Omni article, "MoE 实现的源码级要点":
+// tokens are reordered so that each expert's rows are contiguous before the
+// grouped expert GEMMs).
+//
+// A stable counting sort keyed by expert: row(t, j) = offset[e] + #{t' < t :
+// e in ids[t']} with e = ids[t, j] (a token never holds an expert twice), so
+// rows are ordered by expert, then token -- unique and deterministic.
+//   1. count:   per 32-token warp, one bit per token in a per-expert mask;
+//               block histogram = popcounts of the masks.
+//   2. scan:    one CTA turns the block histograms into per-block row bases
+//               and per-expert offsets (+ the prefix of 128-row GEMM tiles).
+//   3. scatter: rank inside the warp = popcount of the lower lanes' bits.
+//   4. gather:  xp[row] = x[tok_of[row]] (skipped when x is not given).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rmoe {
+
+namespace {
+
+constexpr int PT = PERMUTE_TOK;      // tokens per block (8 warps)
+constexpr int PW = PERMUTE_TOK / 32; // warps per block
+constexpr int MAXE = 128;
+
+__device__ __forceinline__ void build_masks(const int32_t* __restrict__ ids, int T, int E,
+                                            int top_k, uint32_t (*masks)[MAXE], int* status) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < PW * MAXE; i += PT) (&masks[0][0])[i] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * PT + tid;
+  if (t < T) {
+    for (int j = 0; j < top_k; ++j) {
+      const int e = ids[(size_t)t * top_k + j];
+      if (e >= 0 && e < E)
+        atomicOr(&masks[warp][e], 1u << lane);
+      else
+        report_error(status, MOE_ERR_DEVICE_INDEX, 1);
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(PT)
+    permute_count_kernel(const int32_t* __restrict__ ids, int T, int E, int top_k,
+                         int* __restrict__ blk_hist, int* status) {
+  __shared__ uint32_t masks[PW][MAXE];
+  build_masks(ids, T, E, top_k, masks, status);
+  for (int e = threadIdx.x; e < E; e += PT) {
+    int cnt = 0;
+#pragma unroll
+    for (int w = 0; w < PW; ++w) cnt += __popc(masks[w][e]);
+    blk_hist[(size_t)blockIdx.x * E + e] = cnt;
+  }
+}
+
+// One CTA of 1024 threads: expert e = tid % E, chunk ch = tid / E of the blocks.
+__global__ void __launch_bounds__(1024)
+    permute_scan_kernel(int* __restrict__ blk_hist, int nblk, int E,
+                        int* __restrict__ expert_offsets, int* __restrict__ mtile_start) {
+  __shared__ int part[1024];
+  __shared__ int excl_rows[MAXE + 1];
+  __shared__ int excl_tiles[MAXE + 1];
+  const int tid = threadIdx.x;
+  const int C = 1024 / E;
+  const int e = tid % E, ch = tid / E;
+  const bool active = ch < C;
+  int b0 = 0, b1 = 0;
+  if (active) {
+    b0 = (int)((long long)ch * nblk / C);
+    b1 = (int)((long long)(ch + 1) * nblk / C);
+    int s = 0;
+    for (int b = b0; b < b1; ++b) s += blk_hist[(size_t)b * E + e];
+    part[ch * E + e] = s;
+  }
+  __syncthreads();
+  if (tid < 32) {
+    // warp 0: per-expert totals, chunk prefixes, then an exclusive scan over experts
+    int loc_rows[MAXE / 32], loc_tiles[MAXE / 32];
+    int sr = 0, st = 0;
+#pragma unroll
+    for (int q = 0; q < MAXE / 32; ++q) {
+      const int ee = tid * (MAXE / 32) + q;
+      int tot = 0;
+      if (ee < E) {
+        for (int c = 0; c < C; ++c) {
+          const int v = part[c * E + ee];
+          part[c * E + ee] = tot;  // exclusive prefix over chunks
+          tot += v;
+        }
+      }
+      loc_rows[q] = tot;
+      loc_tiles[q] = (tot + MTILE - 1) / MTILE;
+      sr += loc_rows[q];
+      st += loc_tiles[q];
+    }
+    int ir = sr, it = st;  // inclusive warp scan of the per-lane sums
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, ir, off);
+      const int b = __shfl_up_sync(0xffffffffu, it, off);
+      if (tid >= off) {
+        ir += a;
+        it += b;
+      }
+    }
+    int run_r = ir - sr, run_t = it - st;
+#pragma unroll
+    for (int q = 0; q < MAXE / 32; ++q) {
+      const int ee = tid * (MAXE / 32) + q;
+      if (ee < E) {
+        excl_rows[ee] = run_r;
+        excl_tiles[ee] = run_t;
+      }
+      run_r += loc_rows[q];
+      run_t += loc_tiles[q];
+    }
+    if (tid == 31) {
+      excl_rows[E] = ir;
+      excl_tiles[E] = it;
+    }
+  }
+  __syncthreads();
+  if (tid <= E) {
+    expert_offsets[tid] = excl_rows[tid];
+    if (mtile_start) mtile_start[tid] = excl_tiles[tid];
+  }
+  if (active) {
+    int run = excl_rows[e] + part[ch * E + e];
+    for (int b = b0; b < b1; ++b) {
+      const size_t i = (size_t)b * E + e;
+      const int v = blk_hist[i];
+      blk_hist[i] = run;  // base row of expert e inside block b
+      run += v;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(PT)
+    permute_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w,
+                           int T, int E, int top_k, const int* __restrict__ blk_base,
+                           int* __restrict__ row_of, int* __restrict__ tok_of,
+                           float* __restrict__ w_of, int* status) {
+  __shared__ uint32_t masks[PW][MAXE];
+  __shared__ int wbase[PW][MAXE];
+  build_masks(ids, T, E, top_k, masks, status);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < E; e += PT) {
+    int run = blk_base[(size_t)blockIdx.x * E + e];
+#pragma unroll
+    for (int w = 0; w < PW; ++w) {
+      wbase[w][e] = run;
+      run += __popc(masks[w][e]);
+    }
+  }
+  __syncthreads();
+  const int t = blockIdx.x * PT + tid;
+  if (t >= T) return;
+  const uint32_t lower = (1u << lane) - 1u;
+  for (int j = 0; j < top_k; ++j) {
+    const size_t tj = (size_t)t * top_k + j;
+    const int e = ids[tj];
+    if (e < 0 || e >= E) {
+      row_of[tj] = -1;
+      continue;
+    }
+    const int row = wbase[warp][e] + __popc(masks[warp][e] & lower);
+    row_of[tj] = row;
+    tok_of[row] = t;
+    if (w_of) w_of[row] = topk_w ? topk_w[tj] : 1.0f;
+  }
+}
+
+// One warp per destination row; 16-byte vectors.
+__global__ void __launch_bounds__(256)
+    gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int* __restrict__ tok_of,
+                       int R, int H, int T, __nv_bfloat16* __restrict__ xp) {
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += warps) {
+    const int t = tok_of[r];
+    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * H);
+    if (t < 0 || t >= T) {
+      for (int c = lane; c < H / 8; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+    for (int c = lane; c < H / 8; c += 32) dst[c] = src[c];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const void* x, int T,
+                           int H, int E, int top_k, const PermuteOut& o, cudaStream_t stream) {
+  const int nblk = (T + PT - 1) / PT;
+  permute_count_kernel<<<nblk, PT, 0, stream>>>(topk_ids, T, E, top_k, o.blk_hist, o.status);
+  permute_scan_kernel<<<1, 1024, 0, stream>>>(o.blk_hist, nblk, E, o.expert_offsets,
+                                              o.mtile_start);
+  permute_scatter_kernel<<<nblk, PT, 0, stream>>>(topk_ids, topk_w, T, E, top_k, o.blk_hist,
+                                                  o.row_of, o.tok_of, o.w_of, o.status);
+  if (o.xp && x) {
+    const int R = T * top_k;
+    int grid = (R + 7) / 8;
+    const int cap = num_sms() * 16;
+    if (grid > cap) grid = cap;
+    gather_rows_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), o.tok_of,
+                                                 R, H, T, static_cast<__nv_bfloat16*>(o.xp));
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace rmoe

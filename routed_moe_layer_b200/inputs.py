@@ -77,18 +77,18 @@ def make_tokens(T: int, H: int, seed: int, device="cpu") -> torch.Tensor:
 
 def make_weights(H: int, seed: int, E: int = 128, I: int = 768, I_shared: int = 768,
                  device="cpu", layer: int = 0, hot_experts=None, hot_bias: float = 0.5,
-                 weight_std: float = 0.02):
+                 wr_std: float = 0.02, w13_std: float = 0.02, w2_std: float = 0.02):
     """Returns dict(Wr, bias, w13, w2, ws13, ws2) for one block."""
     base = seed * 1000 + 100 * layer
-    Wr = _normal((E, H), 0.02, base + 1, device, torch.float32)
+    Wr = _normal((E, H), wr_std, base + 1, device, torch.float32)
     bias = _uniform((E,), -0.1, 0.1, base + 2, device)
     if hot_experts is not None:
         bias[list(hot_experts)] = hot_bias
-    w13 = _normal((E, 2 * I, H), weight_std, base + 3, device, torch.bfloat16)
-    w2 = _normal((E, H, I), weight_std, base + 4, device, torch.bfloat16)
+    w13 = _normal((E, 2 * I, H), w13_std, base + 3, device, torch.bfloat16)
+    w2 = _normal((E, H, I), w2_std, base + 4, device, torch.bfloat16)
     if I_shared > 0:
-        ws13 = _normal((2 * I_shared, H), weight_std, base + 5, device, torch.bfloat16)
-        ws2 = _normal((H, I_shared), weight_std, base + 6, device, torch.bfloat16)
+        ws13 = _normal((2 * I_shared, H), w13_std, base + 5, device, torch.bfloat16)
+        ws2 = _normal((H, I_shared), w2_std, base + 6, device, torch.bfloat16)
     else:
         ws13 = ws2 = None
     return dict(Wr=Wr, bias=bias, w13=w13, w2=w2, ws13=ws13, ws2=ws2)
@@ -96,10 +96,16 @@ def make_weights(H: int, seed: int, E: int = 128, I: int = 768, I_shared: int = 
 
 def make_block_inputs(T: int, H: int, seed: int, E: int = 128, I: int = 768,
                       I_shared: int = 768, device="cpu", hot_experts=None,
-                      hot_bias: float = 0.5):
-    """Tokens + weights of one block: dict(x, Wr, bias, w13, w2, ws13, ws2)."""
+                      hot_bias: float = 0.5, unit_scale: bool = False):
+    """Tokens + weights of one block: dict(x, Wr, bias, w13, w2, ws13, ws2).
+
+    unit_scale: draw every weight with std 1/sqrt(fan_in) (router included),
+    so that logits, activations and outputs are O(1) at any size."""
+    stds = {}
+    if unit_scale:
+        stds = dict(wr_std=H ** -0.5, w13_std=H ** -0.5, w2_std=I ** -0.5)
     d = make_weights(H, seed, E=E, I=I, I_shared=I_shared, device=device,
-                     hot_experts=hot_experts, hot_bias=hot_bias)
+                     hot_experts=hot_experts, hot_bias=hot_bias, **stds)
     d["x"] = make_tokens(T, H, seed, device=device)
     return d
 

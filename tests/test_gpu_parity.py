@@ -1,0 +1,273 @@
+"""CUDA path (through the C ABI) against the CPU oracle.
+
+Sizes span several 128-row tiles with ragged tails, experts with no tokens,
+N tails (I and H not multiples of the tile), T = 1, the skewed (hot expert)
+case, the named workloads (the two small ones in full, the large ones on a
+seeded token sample), determinism and batch isolation.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from routed_moe_layer_b200 import inputs, ops
+from routed_moe_layer_b200.ops import BlockConfig
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _dev(d):
+    return {k: (None if v is None else v.to(DEV)) for k, v in d.items()}
+
+
+def _run(d, cfg, residual=None):
+    ids = torch.empty((cfg.T, cfg.top_k), dtype=torch.int32, device=DEV)
+    w = torch.empty((cfg.T, cfg.top_k), dtype=torch.float32, device=DEV)
+    ws = ops.alloc_workspace(ops.workspace_bytes(cfg), DEV)
+    out = ops.forward(d["x"], d["Wr"], d["bias"], d["w13"], d["w2"], d.get("ws13"), d.get("ws2"),
+                      cfg, residual=residual, workspace=ws, topk_ids=ids, topk_w=w)
+    torch.cuda.synchronize()
+    code, site = ops.read_device_status(ws)
+    assert code == 0, (ops.status_string(code), site)
+    return out, ids, w
+
+
+# ------------------------------------------------------------------ router
+@pytest.mark.parametrize("T,H,E,k,G,g", [
+    (1, 64, 8, 2, 4, 2), (37, 128, 16, 4, 4, 2), (300, 256, 128, 8, 4, 2),
+    (1000, 1024, 128, 8, 4, 2), (129, 2048, 64, 6, 8, 3), (50, 512, 32, 4, 1, 1),
+    (65, 192, 96, 16, 4, 4),
+])
+def test_router_matches_oracle(T, H, E, k, G, g):
+    cfg = BlockConfig(T=T, H=H, E=E, top_k=k, n_group=G, topk_group=g)
+    d = inputs.make_block_inputs(T, H, seed=T + E, E=E, I=64, I_shared=0, unit_scale=True)
+    dd = _dev(d)
+    ids, w = ops.route(dd["x"], dd["Wr"], dd["bias"], cfg)
+    torch.cuda.synchronize()
+    rep = parity.check_routing(ids, w, *[parity.to_np(d[n]) for n in ("x", "Wr", "bias")], cfg)
+    assert rep["near_ties"] <= max(2, T // 20)
+
+
+@pytest.mark.parametrize("wid", [0, 1, 2, 3])
+def test_router_on_workloads(wid):
+    wl = inputs.WORKLOADS[wid]
+    d = inputs.workload_inputs(wid)
+    cfg = BlockConfig(T=wl.T, H=wl.H)
+    dd = {k: d[k].to(DEV) for k in ("x", "Wr", "bias")}
+    ids, w = ops.route(dd["x"], dd["Wr"], dd["bias"], cfg)
+    torch.cuda.synchronize()
+    rep = parity.check_routing(ids, w, *[parity.to_np(d[n]) for n in ("x", "Wr", "bias")], cfg)
+    print(f"workload {wl.name}: {rep}")
+    # weights sum to the scaling factor on every token
+    np.testing.assert_allclose(w.sum(1).cpu().numpy(), 2.5, rtol=1e-5)
+
+
+def test_router_bias_forces_selection_not_weights():
+    T, H = 200, 512
+    cfg = BlockConfig(T=T, H=H)
+    d = _dev(inputs.make_block_inputs(T, H, seed=5, I=64, I_shared=0, unit_scale=True))
+    forced = [3, 7, 40, 41, 44, 60, 61, 63]  # groups 0 and 1 only
+    b = d["bias"].clone()
+    b[forced] += 10.0
+    ids, w = ops.route(d["x"], d["Wr"], b, cfg)
+    ids0, w0 = ops.route(d["x"], d["Wr"], d["bias"], cfg)
+    assert all(sorted(r) == forced for r in ids.cpu().tolist())
+    # same ids -> bitwise the same weights whatever the bias
+    same = (torch.sort(ids, 1).values == torch.sort(ids0, 1).values).all(1)
+    for t in torch.nonzero(same).flatten().tolist():
+        o, o0 = torch.argsort(ids[t]), torch.argsort(ids0[t])
+        assert torch.equal(w[t][o], w0[t][o0])
+
+
+# ------------------------------------------------------------------ permutation
+@pytest.mark.parametrize("T,E,k", [(1, 8, 2), (255, 128, 8), (256, 128, 8), (257, 128, 8),
+                                   (1000, 16, 4), (19412, 128, 8)])
+def test_permute_bit_exact(T, E, k):
+    g = torch.Generator().manual_seed(T * 7 + E)
+    ids = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
+    w = torch.rand((T, k), generator=g)
+    H = 128
+    x = torch.randn((T, H), generator=g).to(torch.bfloat16)
+    cfg = BlockConfig(T=T, H=H, E=E, top_k=k, n_group=1, topk_group=1)
+    r = ops.permute(ids.to(DEV), cfg, topk_w=w.to(DEV), x=x.to(DEV))
+    torch.cuda.synchronize()
+    code, _ = ops.read_device_status(r["workspace"])
+    assert code == 0
+    off, row_of, tok_of = oracle.permutation(ids.numpy(), E)
+    assert np.array_equal(r["expert_offsets"].cpu().numpy(), off)
+    assert np.array_equal(r["row_of"].cpu().numpy(), row_of)
+    assert np.array_equal(r["tok_of"].cpu().numpy(), tok_of)
+    assert torch.equal(r["w_of"].cpu(), w.reshape(-1)[torch.as_tensor(np.argsort(row_of))])
+    assert torch.equal(r["xp"].cpu(), x[torch.as_tensor(tok_of)])
+
+
+def test_permute_reports_bad_expert_id():
+    T, E, k = 64, 16, 2
+    ids = torch.tensor([[i % E, (i + 1) % E] for i in range(T)], dtype=torch.int32)
+    ids[5, 1] = E  # out of range: skipped and reported
+    cfg = BlockConfig(T=T, H=64, E=E, top_k=k, n_group=1, topk_group=1)
+    r = ops.permute(ids.to(DEV), cfg)
+    torch.cuda.synchronize()
+    code, site = ops.read_device_status(r["workspace"])
+    assert code == 6  # MOE_ERR_DEVICE_INDEX
+    assert r["row_of"][5 * k + 1].item() == -1
+
+
+# ------------------------------------------------------------------ forward
+FORWARD_CASES = [
+    # T, H, E, I, I_shared, k, G, g
+    (1, 256, 16, 128, 128, 4, 4, 2),
+    (100, 256, 16, 128, 128, 4, 4, 2),
+    (300, 512, 32, 192, 64, 8, 4, 2),       # I not a multiple of 128: SwiGLU N tail
+    (700, 320, 16, 128, 128, 4, 4, 2),      # H not a multiple of 256: down/combine N tail
+    (1000, 1024, 128, 768, 768, 8, 4, 2),   # several tiles per expert, ragged tails
+    (2048, 2048, 128, 768, 768, 8, 4, 2),
+]
+
+
+@pytest.mark.parametrize("T,H,E,I,Is,k,G,g", FORWARD_CASES)
+def test_forward_matches_oracle(T, H, E, I, Is, k, G, g):
+    cfg = BlockConfig(T=T, H=H, E=E, I=I, I_shared=Is, top_k=k, n_group=G, topk_group=g)
+    d = inputs.make_block_inputs(T, H, seed=11 + T, E=E, I=I, I_shared=Is, unit_scale=True)
+    out, ids, w = _run(_dev(d), cfg)
+    dn = parity.np_inputs(d)
+    parity.check_routing(ids, w, dn["x"], dn["Wr"], dn["bias"], cfg)
+    rep = parity.check_output(out, ids, dn, cfg)
+    assert rep["rms_rel"] < 1e-2, rep  # bf16 storage of h and Y: a few 1e-3
+
+
+def test_forward_residual_and_no_shared_expert():
+    T, H, E, I = 513, 512, 32, 128
+    for Is in (0, 128):
+        cfg = BlockConfig(T=T, H=H, E=E, I=I, I_shared=Is)
+        d = inputs.make_block_inputs(T, H, seed=3, E=E, I=I, I_shared=Is, unit_scale=True)
+        dd = _dev(d)
+        res = torch.randn((T, H), generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+        out, ids, _ = _run(dd, cfg, residual=res.to(DEV))
+        rep = parity.check_output(out, ids, parity.np_inputs(d), cfg,
+                                  residual_np=parity.to_np(res))
+        assert rep["rms_rel"] < 1e-2, rep
+
+
+def test_forward_in_place_residual():
+    T, H = 300, 256
+    cfg = BlockConfig(T=T, H=H, E=16, I=128, I_shared=128, top_k=4)
+    d = _dev(inputs.make_block_inputs(T, H, seed=8, E=16, I=128, I_shared=128, unit_scale=True))
+    res = torch.randn((T, H), device=DEV).to(torch.bfloat16)
+    ref = ops.forward(d["x"], d["Wr"], d["bias"], d["w13"], d["w2"], d["ws13"], d["ws2"], cfg,
+                      residual=res)
+    buf = res.clone()
+    ops.forward(d["x"], d["Wr"], d["bias"], d["w13"], d["w2"], d["ws13"], d["ws2"], cfg,
+                residual=buf, out=buf)
+    torch.cuda.synchronize()
+    assert torch.equal(buf, ref)
+
+
+def test_forward_hot_experts_many_tiles():
+    # a bias of +10 on 8 experts (2 groups) sends every token to them: those
+    # experts get T rows (many full tiles + a tail), the other 120 get none
+    T, H = 1500, 512
+    cfg = BlockConfig(T=T, H=H, I=256, I_shared=128)
+    d = inputs.make_block_inputs(T, H, seed=21, I=256, I_shared=128, unit_scale=True)
+    hot = [0, 5, 9, 31, 64, 70, 80, 95]
+    d["bias"][hot] += 10.0
+    out, ids, w = _run(_dev(d), cfg)
+    assert all(sorted(r) == hot for r in ids.cpu().tolist())
+    rep = parity.check_output(out, ids, parity.np_inputs(d), cfg)
+    assert rep["rms_rel"] < 1e-2, rep
+
+
+@pytest.mark.parametrize("wid", [0, 1])
+def test_forward_small_workloads_in_full(wid):
+    wl = inputs.WORKLOADS[wid]
+    cfg = BlockConfig(T=wl.T, H=wl.H)
+    d = inputs.workload_inputs(wid)
+    out, ids, w = _run(_dev(d), cfg)
+    dn = parity.np_inputs(d)
+    rrep = parity.check_routing(ids, w, dn["x"], dn["Wr"], dn["bias"], cfg)
+    orep = parity.check_output(out, ids, dn, cfg)
+    print(f"{wl.name}: routing {rrep} output {orep}")
+    assert orep["rms_rel"] < 1e-2
+
+
+@pytest.mark.parametrize("wid", [2, 3])
+def test_forward_large_workloads_sampled(wid):
+    wl = inputs.WORKLOADS[wid]
+    cfg = BlockConfig(T=wl.T, H=wl.H)
+    d = inputs.workload_inputs(wid)
+    out, ids, w = _run(_dev(d), cfg)
+    dn = parity.np_inputs(d)
+    rrep = parity.check_routing(ids, w, dn["x"], dn["Wr"], dn["bias"], cfg)
+    rng = np.random.default_rng(wid)
+    sample = np.concatenate([[0, wl.T - 1], rng.choice(wl.T, 254, replace=False)])
+    orep = parity.check_output(out, ids, dn, cfg, tokens=sample)
+    counts = np.bincount(ids.cpu().numpy().ravel(), minlength=128)
+    print(f"{wl.name}: routing {rrep} output {orep} rows/expert min {counts.min()} "
+          f"max {counts.max()}")
+    assert orep["rms_rel"] < 1e-2
+    if wl.hot_experts is not None:
+        frac = counts[list(wl.hot_experts)].sum() / counts.sum()
+        print(f"hot-expert share of selections: {frac:.3f}")
+
+
+def test_forward_deterministic_and_isolated():
+    T, H = 1000, 1024
+    cfg = BlockConfig(T=T, H=H)
+    d = _dev(inputs.make_block_inputs(T, H, seed=99, unit_scale=True))
+    a, ids_a, _ = _run(d, cfg)
+    b, ids_b, _ = _run(d, cfg)
+    assert torch.equal(a, b) and torch.equal(ids_a, ids_b)
+    # each token's output does not depend on the other tokens of the call
+    split = 371
+    for lo, hi in ((0, split), (split, T)):
+        part = dict(d, x=d["x"][lo:hi].contiguous())
+        p, _, _ = _run(part, cfg.with_tokens(hi - lo))
+        assert torch.equal(p, a[lo:hi])
+
+
+# ------------------------------------------------------------------ RMSNorm, residual stack
+def test_rmsnorm_matches_oracle():
+    T, H = 333, 2048
+    x = (3.0 * torch.randn((T, H), generator=torch.Generator().manual_seed(4))).to(torch.bfloat16)
+    gamma = torch.rand(H, generator=torch.Generator().manual_seed(5)) + 0.5
+    for g in (None, gamma):
+        y = ops.rmsnorm(x.to(DEV), None if g is None else g.to(DEV), eps=1e-6)
+        ref = oracle.rmsnorm(parity.to_np(x), 1e-6, None if g is None else g.numpy())
+        got = parity.to_np(y)
+        # one bf16 rounding of an fp32 result
+        assert np.max(np.abs(got - ref) / (np.abs(ref) + 1e-3)) < 8e-3
+
+
+def test_residual_stack_teacher_forced():
+    # x <- x + block_l(RMSNorm(x)) for 3 layers; each layer is checked against
+    # the oracle on the GPU's own bf16 input to that layer
+    T, H, L = 700, 1024, 3
+    cfg = BlockConfig(T=T, H=H)
+    x = inputs.make_tokens(T, H, seed=4).to(DEV)
+    for layer in range(L):
+        wts = inputs.make_weights(H, seed=4, layer=layer)
+        dw = _dev(wts)
+        xin = x.clone()
+        xn = ops.rmsnorm(x, eps=1e-6)
+        out, ids, w = _run(dict(dw, x=xn), cfg, residual=x)
+        dn = parity.np_inputs(dict(wts, x=xn.cpu()))
+        parity.check_routing(ids, w, dn["x"], dn["Wr"], dn["bias"], cfg)
+        rep = parity.check_output(out, ids, dn, cfg, residual_np=parity.to_np(xin))
+        assert rep["rms_rel"] < 1e-2
+        x = out
+
+
+# ------------------------------------------------------------------ failure detection
+def test_bounded_wait_times_out_and_context_survives():
+    code, site = ops.selftest_wait_timeout(timeout_ns=50_000_000)  # 50 ms
+    assert code == 5 and site == 99
+    # the context is still usable
+    T, H = 64, 256
+    cfg = BlockConfig(T=T, H=H, E=16, I=128, I_shared=128, top_k=4)
+    d = _dev(inputs.make_block_inputs(T, H, seed=1, E=16, I=128, I_shared=128, unit_scale=True))
+    out, ids, _ = _run(d, cfg)
+    assert torch.isfinite(out.float()).all()

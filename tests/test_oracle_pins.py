@@ -16,7 +16,7 @@ import pytest
 import torch
 
 from oracle import (MoeConfig, bf16_round, group_limited_topk, moe_forward,
-                    moe_forward_tokens, rmsnorm, route, router_scores,
+                    moe_forward_tokens, permutation, rmsnorm, route, router_scores,
                     routing_weights, swiglu_mlp)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -308,3 +308,20 @@ def test_invalid_configs_raise():
         group_limited_topk(c, 4, 2, 2)  # 10 % 4 != 0
     with pytest.raises(ValueError):
         group_limited_topk(np.zeros((1, 8), np.float32), 4, 1, 3)  # 2 candidates < 3
+
+
+def test_permutation_matches_counting_definition():
+    # row(t, j) = offset[e] + #{t' < t : e in ids[t']}, e = ids[t, j]; offsets = prefix counts
+    rng = np.random.default_rng(17)
+    T, E, k = 57, 12, 3
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    offsets, row_of, tok_of = permutation(ids, E)
+    counts = [int((ids == e).sum()) for e in range(E)]
+    assert offsets.tolist() == [sum(counts[:e]) for e in range(E + 1)]
+    for t in range(T):
+        for j in range(k):
+            e = ids[t, j]
+            before = sum(1 for tp in range(t) if e in ids[tp])
+            r = offsets[e] + before
+            assert row_of[t * k + j] == r and tok_of[r] == t
+    assert sorted(row_of.tolist()) == list(range(T * k))
