@@ -36,6 +36,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from routed_moe_layer_b200 import inputs, ops  # noqa: E402
+from routed_moe_layer_b200.dist import max_over_ranks, rank_token_seed  # noqa: E402
 from routed_moe_layer_b200.ops import BlockConfig  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and TFLOP/s at T~19.4k bf16; % of roofline"
@@ -137,11 +138,7 @@ def _barrier(world):
 
 
 def _max_over_ranks(v: float, world: int) -> float:
-    if world == 1:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+    return max_over_ranks(v) if world > 1 else v
 
 
 def cpu_oracle_sample(cfg_id: int, target_s: float = 12.0, d_cpu=None):
@@ -243,7 +240,7 @@ def run_ours(args, world, rank, local):
         wd = inputs.make_weights(wl.H, wl.seed, device=gen_dev, layer=l,
                                  hot_experts=wl.hot_experts, hot_bias=wl.hot_bias)
         weights.append({k: (None if v is None else v.to(dev)) for k, v in wd.items()})
-    x_host = inputs.make_tokens(wl.T, wl.H, wl.seed + 1000 * rank).pin_memory()
+    x_host = inputs.make_tokens(wl.T, wl.H, rank_token_seed(wl.seed, rank)).pin_memory()
     x = x_host.to(dev)
     ws = ops.alloc_workspace(ops.workspace_bytes(cfg), dev)
     out = torch.empty_like(x)

@@ -201,7 +201,12 @@ class StageTimer:
 
     def __init__(self):
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(NUM_STAGES + 1)]
-        self._arr = (ctypes.c_void_p * (NUM_STAGES + 1))(*[e.cuda_event for e in self.events])
+        for e in self.events:  # torch creates the CUDA event on its first record
+            e.record()
+        handles = [e.cuda_event for e in self.events]
+        if not all(handles):
+            raise RuntimeError("could not create CUDA events for stage timing")
+        self._arr = (ctypes.c_void_p * (NUM_STAGES + 1))(*handles)
 
     def as_ptr(self):
         return ctypes.cast(self._arr, ctypes.POINTER(ctypes.c_void_p))
