@@ -56,6 +56,24 @@ def algorithmic_bytes(cfg: BlockConfig, experts_used: int) -> float:
             cfg.E * 4 + 2.0 * cfg.T * cfg.H * 2)
 
 
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of ``kernel`` from the committed ncu summary, or None when the
+    kernel's source has changed since the counters were taken (or none were taken)."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel)
+    if not rec or rec.get("workload") != workload:
+        return None
+    with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if not sha.startswith(rec["source_sha256_prefix"]):
+        return None
+    return float(rec["dram_bytes_read"] + rec["dram_bytes_write"])
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -331,7 +349,8 @@ def run_ours(args, world, rank, local):
               "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
               "frac": achieved / peak_tf,
               "peak_source": f"{peak_src} bf16 dense burst",
-              "traffic": None,
+              "traffic": measured_traffic("grouped_gemm_kernel<EPI_SWIGLU>", wl.name),
+              "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
               "layer_roofline_frac": max(fpt * wl.T / peak_tf / 1e12,
                                          hbm_bytes / peaks["hbm_gbs"] / 1e9) / (layer_ms * 1e-3)}
         cpu_tps, cores, sample = (None, None, None)
