@@ -142,6 +142,32 @@ MOE_API int32_t moe_permute(const int32_t* topk_ids, const float* topk_w, const 
                     int32_t* tok_of, float* w_of, void* xp, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/* Largest T that moe_permute_noalloc accepts. */
+#define MOE_NOALLOC_MAX_T 65536
+
+/* moe_permute without a workspace argument: the same permutation, bit for
+ * bit, for callers that cannot allocate device memory themselves -- for
+ * example an operator running inside another framework that hands it its
+ * inputs and outputs and owns every device allocation, or a latency-critical
+ * loop where a cudaMalloc (which can synchronise the device) is not allowed.
+ * The source pages have no counterpart to this entry point.
+ *   Arguments are those of moe_permute minus workspace / workspace_bytes.
+ *   Scratch: a fixed array of about 129 KiB in the library's device memory,
+ *   one copy on every GPU that loads the library, held until the process
+ *   exits.  T > MOE_NOALLOC_MAX_T returns MOE_ERR_UNSUPPORTED_SHAPE and
+ *   launches nothing.  The call allocates nothing (no cudaMalloc/cudaFree).
+ *   The first call on a device looks up the array's device address (once
+ *   per device, with that device current); make that first call before any
+ *   stream capture.
+ *   Every call on a device shares the one array and it keeps the last call's
+ *   contents: calls that overlap on the GPU (different streams, no ordering)
+ *   race and give wrong results.  An expert id outside [0,E) is skipped and
+ *   its row_of entry set to -1 (the status word is not exposed). */
+MOE_API int32_t moe_permute_noalloc(const int32_t* topk_ids, const float* topk_w, const void* x,
+                                    const moe_cfg_t* cfg, int32_t* expert_offsets,
+                                    int32_t* row_of, int32_t* tok_of, float* w_of, void* xp,
+                                    void* stream);
+
 /* Whole block forward ([S1] LingBotVideoSparseMoeBlock.forward: router ->
  * grouped SwiGLU experts with the router weight applied on the output ->
  * fp32 restore ([S2] "_restore_tokens") -> + shared expert, unscaled).

@@ -1,0 +1,75 @@
+"""The allocation-free permutation entry point, through the C ABI.
+
+moe_permute_noalloc is for callers that may not allocate device memory
+themselves (an operator inside another framework that owns all device
+memory; a latency-critical loop where cudaMalloc is not allowed).  Its
+scratch is a fixed array inside the library, so this test checks that two
+calls in a row -- the second one seeing the first one's leftovers -- each
+give exactly what the workspace-taking moe_permute gives.
+"""
+
+import ctypes
+
+import pytest
+import torch
+
+from routed_moe_layer_b200 import ops
+from routed_moe_layer_b200.ops import BlockConfig
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _noalloc_fn():
+    f = ops.lib().moe_permute_noalloc
+    vp = ctypes.c_void_p
+    f.restype = ctypes.c_int32
+    f.argtypes = [vp, vp, vp, ctypes.POINTER(ops.MoeCfg), vp, vp, vp, vp, vp, vp]
+    return f
+
+
+def _inputs(T, E, k, H, seed):
+    g = torch.Generator().manual_seed(seed)
+    ids = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
+    w = torch.rand((T, k), generator=g)
+    x = torch.randn((T, H), generator=g).to(torch.bfloat16)
+    return ids.to(DEV), w.to(DEV), x.to(DEV)
+
+
+def _noalloc(ids, w, x, cfg):
+    T, k, E = cfg.T, cfg.top_k, cfg.E
+    offsets = torch.full((E + 1,), -7, dtype=torch.int32, device=DEV)
+    row_of = torch.full((T * k,), -7, dtype=torch.int32, device=DEV)
+    tok_of = torch.full((T * k,), -7, dtype=torch.int32, device=DEV)
+    w_of = torch.zeros(T * k, dtype=torch.float32, device=DEV)
+    xp = torch.zeros((T * k, cfg.H), dtype=torch.bfloat16, device=DEV)
+    c = cfg.c()
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    code = _noalloc_fn()(p(ids), p(w), p(x), ctypes.byref(c), p(offsets), p(row_of), p(tok_of),
+                         p(w_of), p(xp),
+                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert code == 0, ops.status_string(code)
+    torch.cuda.synchronize()
+    return dict(expert_offsets=offsets, row_of=row_of, tok_of=tok_of, w_of=w_of, xp=xp)
+
+
+def test_noalloc_permute_matches_workspace_permute_twice():
+    # the second call has fewer tokens and another expert count, so stale
+    # histogram rows of the first call would show up if they were read
+    for T, E, k, seed in ((5000, 128, 8, 1), (1234, 64, 6, 2)):
+        cfg = BlockConfig(T=T, H=256, E=E, top_k=k, n_group=1, topk_group=1)
+        ids, w, x = _inputs(T, E, k, cfg.H, seed)
+        got = _noalloc(ids, w, x, cfg)
+        ref = ops.permute(ids, cfg, topk_w=w, x=x)
+        torch.cuda.synchronize()
+        for name in ("expert_offsets", "row_of", "tok_of", "w_of", "xp"):
+            assert torch.equal(got[name], ref[name]), name
+
+
+def test_noalloc_rejects_tokens_beyond_its_scratch():
+    cfg = BlockConfig(T=65537, H=256, E=128, top_k=8, n_group=1, topk_group=1)
+    c = cfg.c()
+    fake = ctypes.c_void_p(0x10000)  # never dereferenced: the size check fails first
+    code = _noalloc_fn()(fake, None, None, ctypes.byref(c), fake, fake, fake, None, None, None)
+    assert code == 2  # MOE_ERR_UNSUPPORTED_SHAPE
