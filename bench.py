@@ -41,7 +41,7 @@ from routed_moe_layer_b200.ops import BlockConfig  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and TFLOP/s at T~19.4k bf16; % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 9  # router, 3 permute, gather, expert up, expert down, shared up, combine
+KERNELS_PER_STEP = 12  # router 3, permute 3 + gather, expert up/down, shared up/down, combine
 
 
 def flops_per_token(cfg: BlockConfig) -> float:

@@ -83,7 +83,7 @@ typedef struct {
 #define MOE_STAGE_PERMUTE 1
 #define MOE_STAGE_EXPERT_UP 2
 #define MOE_STAGE_EXPERT_DOWN 3
-#define MOE_STAGE_SHARED_UP 4
+#define MOE_STAGE_SHARED_EXPERT 4
 #define MOE_STAGE_COMBINE 5
 #define MOE_NUM_STAGES 6
 
@@ -119,7 +119,8 @@ MOE_API size_t moe_workspace_bytes(const moe_cfg_t* cfg);
  *   bias     device fp32 [E]     e_score_correction_bias (selection only)
  *   topk_ids device int32 [T,top_k] out: expert ids, descending c, ties to the lower id
  *   topk_w   device fp32 [T,top_k] out: gating weights, same order
- *   workspace may be NULL when moe_route_workspace_bytes(cfg) == 0. */
+ *   workspace device, moe_route_workspace_bytes(cfg) bytes, 256-byte aligned:
+ *            status word, the bf16 three-term split of Wr and fp32 partial logits. */
 MOE_API int32_t moe_route(const void* x, const float* Wr, const float* bias, const moe_cfg_t* cfg,
                   int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes,
                   void* stream);
@@ -178,10 +179,11 @@ MOE_API int32_t moe_permute_noalloc(const int32_t* topk_ids, const float* topk_w
  *   ws13  device bf16 [2I_s,H], ws2 device bf16 [H,I_s]  (NULL when I_shared == 0)
  *   out   device bf16 [T,H]          must not overlap x
  *   opts  host pointer or NULL
- * The result is rounded to bf16 once, after an fp32 sum in a fixed order
- * (slots 0..top_k-1, then the shared expert, then the residual), so it is
- * bitwise reproducible and each token's output does not depend on the
- * other tokens of the call. */
+ * Each expert output (router weight applied in fp32) is stored as bf16; the
+ * restore sums them in fp32 in a fixed order (slots 0..top_k-1, then the
+ * shared expert, then the residual) and rounds once, so the result is
+ * bitwise reproducible and each token's output does not depend on the other
+ * tokens of the call. */
 MOE_API int32_t moe_forward(const void* x, const float* Wr, const float* bias, const void* w13,
                     const void* w2, const void* ws13, const void* ws2, const moe_cfg_t* cfg,
                     void* out, const moe_forward_opts_t* opts, void* workspace,

@@ -48,8 +48,13 @@ int32_t check_cfg(const moe_cfg_t* c) {
 }
 
 struct FwdLayout {
-  size_t status, ids, w, blk_hist, offsets, mtiles, row_of, tok_of, w_of, xp, h, hs, total;
+  size_t status, router, ids, w, blk_hist, offsets, mtiles, row_of, tok_of, w_of, pos_of, y, h,
+      hs, total;
 };
+
+// Slots per token of the token-major buffer of weighted expert outputs: the
+// routed experts, then the shared expert.
+int slots_per_token(const moe_cfg_t& c) { return c.top_k + (c.I_shared > 0 ? 1 : 0); }
 
 FwdLayout fwd_layout(const moe_cfg_t& c) {
   FwdLayout L;
@@ -57,6 +62,7 @@ FwdLayout fwd_layout(const moe_cfg_t& c) {
   const size_t nblk = (T + PERMUTE_TOK - 1) / PERMUTE_TOK;
   size_t off = 0;
   L.status = off;   off += align_up(sizeof(DevStatus));
+  L.router = off;   off += align_up(router_scratch_bytes(c.T, c.H, c.E));
   L.ids = off;      off += align_up(R * 4);
   L.w = off;        off += align_up(R * 4);
   L.blk_hist = off; off += align_up(nblk * E * 4);
@@ -65,7 +71,10 @@ FwdLayout fwd_layout(const moe_cfg_t& c) {
   L.row_of = off;   off += align_up(R * 4);
   L.tok_of = off;   off += align_up(R * 4);
   L.w_of = off;     off += align_up(R * 4);
-  L.xp = off;       off += align_up(R * c.H * 2);  // gathered rows; reused for weighted outputs
+  L.pos_of = off;   off += align_up(R * 4);
+  // gathered expert rows [R, H]; once the up projection has read them, the same
+  // bytes hold the weighted expert outputs in token-major slot order [T*slots, H]
+  L.y = off;        off += align_up(std::max(R, T * (size_t)slots_per_token(c)) * c.H * 2);
   L.h = off;        off += align_up(R * c.I * 2);
   L.hs = off;       off += align_up(T * c.I_shared * 2);
   L.total = off;
@@ -140,8 +149,8 @@ const char* moe_status_string(int32_t status) {
 int32_t moe_check_config(const moe_cfg_t* cfg) { return check_cfg(cfg); }
 
 size_t moe_route_workspace_bytes(const moe_cfg_t* cfg) {
-  (void)cfg;
-  return 0;
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return align_up(sizeof(DevStatus)) + align_up(router_scratch_bytes(cfg->T, cfg->H, cfg->E));
 }
 
 size_t moe_permute_workspace_bytes(const moe_cfg_t* cfg) {
@@ -159,12 +168,15 @@ int32_t moe_route(const void* x, const float* Wr, const float* bias, const moe_c
                   void* stream) {
   const int32_t st = check_cfg(cfg);
   if (st != MOE_OK) return st;
-  (void)workspace;
-  (void)workspace_bytes;
   if (cfg->T == 0) return MOE_OK;
   if (!x || !Wr || !bias || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!ws_ok(workspace, workspace_bytes, moe_route_workspace_bytes(cfg))) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = at<int>(workspace, 0);
+  RMOE_TRY(launch_status_reset(status, s));
   return cuda_status(launch_router(x, Wr, bias, router_params(*cfg), topk_ids, topk_w,
-                                   static_cast<cudaStream_t>(stream)));
+                                   at<void>(workspace, align_up(sizeof(DevStatus))), status,
+                                   DEFAULT_TIMEOUT_NS, s));
 }
 
 int32_t moe_permute(const int32_t* topk_ids, const float* topk_w, const void* x,
@@ -220,18 +232,20 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
   int* offsets = at<int>(workspace, L.offsets);
   int* mtiles = at<int>(workspace, L.mtiles);
   int* row_of = at<int>(workspace, L.row_of);
-  __nv_bfloat16* xp = at<__nv_bfloat16>(workspace, L.xp);
+  __nv_bfloat16* xp = at<__nv_bfloat16>(workspace, L.y);  // gathered rows, then ...
+  __nv_bfloat16* Y = xp;  // ... token-major weighted outputs (after the up projection)
   __nv_bfloat16* h = at<__nv_bfloat16>(workspace, L.h);
   __nv_bfloat16* hs = at<__nv_bfloat16>(workspace, L.hs);
 
   // tensor maps (host-side descriptors, passed by value to the kernels)
+  const int slots = slots_per_token(c);
   CUtensorMap tm_xp, tm_w13, tm_h, tm_w2, tm_x, tm_ws13, tm_hs, tm_ws2;
   RMOE_TRY(make_tmap_2d(&tm_xp, xp, R, c.H));
+  RMOE_TRY(make_tmap_2d(&tm_x, x, T, c.H));
   RMOE_TRY(make_tmap_3d(&tm_w13, w13, c.E, 2 * (uint64_t)c.I, c.H));
   RMOE_TRY(make_tmap_2d(&tm_h, h, R, c.I));
   RMOE_TRY(make_tmap_3d(&tm_w2, w2, c.E, c.H, c.I));
   if (c.I_shared > 0) {
-    RMOE_TRY(make_tmap_2d(&tm_x, x, T, c.H));
     RMOE_TRY(make_tmap_3d(&tm_ws13, ws13, 1, 2 * (uint64_t)c.I_shared, c.H));
     RMOE_TRY(make_tmap_2d(&tm_hs, hs, T, c.I_shared));
     RMOE_TRY(make_tmap_3d(&tm_ws2, ws2, 1, c.H, c.I_shared));
@@ -244,7 +258,8 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
 
   RMOE_TRY(record(MOE_STAGE_ROUTER));
   RMOE_TRY(launch_status_reset(status, s));
-  RMOE_TRY(launch_router(x, Wr, bias, router_params(c), ids, tw, s));
+  RMOE_TRY(launch_router(x, Wr, bias, router_params(c), ids, tw, at<void>(workspace, L.router),
+                         status, timeout, s));
 
   RMOE_TRY(record(MOE_STAGE_PERMUTE));
   PermuteOut o;
@@ -255,6 +270,8 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
   o.row_of = row_of;
   o.tok_of = at<int>(workspace, L.tok_of);
   o.w_of = at<float>(workspace, L.w_of);
+  o.pos_of = at<int>(workspace, L.pos_of);
+  o.slot_stride = slots;
   o.xp = xp;
   RMOE_TRY(launch_permute(ids, tw, x, c.T, c.H, c.E, c.top_k, o, s));
 
@@ -281,7 +298,7 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
     RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_xp, tm_w13, g, grid, s));
   }
   RMOE_TRY(record(MOE_STAGE_EXPERT_DOWN));
-  {  // Y = w_row * (h . W2^T), per expert, written over the gathered rows
+  {  // Y[t*slots + j] = w_tj * (h . W2^T), per expert
     GemmArgs g = a;
     g.mtile_start = mtiles;
     g.row_start = offsets;
@@ -290,52 +307,48 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
     g.k_steps = c.I / 64;
     g.n_out_tile = 256;
     g.b_second = 128;
-    g.out = xp;
+    g.out = Y;
     g.ldo = c.H;
     g.n_valid = c.H;
     g.row_scale = o.w_of;
+    g.dest_pos = o.pos_of;
     const int grid = (int)std::min<long long>(sms, (long long)mt_bound * g.n_tiles);
     RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, g, grid, s));
   }
-  RMOE_TRY(record(MOE_STAGE_SHARED_UP));
-  const void* residual = opts ? opts->residual : nullptr;
+  RMOE_TRY(record(MOE_STAGE_SHARED_EXPERT));
   if (c.I_shared > 0) {
-    GemmArgs g = a;
-    g.single_rows = c.T;
-    g.n_tiles = (c.I_shared + 127) / 128;
-    g.k_steps = c.H / 64;
-    g.n_out_tile = 128;
-    g.b_second = c.I_shared;
-    g.out = hs;
-    g.ldo = c.I_shared;
-    g.n_valid = c.I_shared;
-    const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
-    RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_x, tm_ws13, g, std::min(sms, tiles), s));
+    {  // hs = silu(x . Ws13g^T) * (x . Ws13u^T)
+      GemmArgs g = a;
+      g.single_rows = c.T;
+      g.n_tiles = (c.I_shared + 127) / 128;
+      g.k_steps = c.H / 64;
+      g.n_out_tile = 128;
+      g.b_second = c.I_shared;
+      g.out = hs;
+      g.ldo = c.I_shared;
+      g.n_valid = c.I_shared;
+      const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
+      RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_x, tm_ws13, g, std::min(sms, tiles), s));
+    }
+    {  // Y[t*slots + top_k] = hs . Ws2^T  (unscaled)
+      GemmArgs g = a;
+      g.single_rows = c.T;
+      g.n_tiles = (c.H + 255) / 256;
+      g.k_steps = c.I_shared / 64;
+      g.n_out_tile = 256;
+      g.b_second = 128;
+      g.out = Y;
+      g.ldo = c.H;
+      g.n_valid = c.H;
+      g.dest_mul = slots;
+      g.dest_add = c.top_k;
+      const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
+      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_hs, tm_ws2, g, std::min(sms, tiles), s));
+    }
   }
   RMOE_TRY(record(MOE_STAGE_COMBINE));
-  if (c.I_shared > 0) {
-    // out = bf16( sum_j Y[row_of[t,j]] + hs . Ws2^T [+ residual] )
-    GemmArgs g = a;
-    g.single_rows = c.T;
-    g.n_tiles = (c.H + 255) / 256;
-    g.k_steps = c.I_shared / 64;
-    g.n_out_tile = 256;
-    g.b_second = 128;
-    g.out = static_cast<__nv_bfloat16*>(out);
-    g.ldo = c.H;
-    g.n_valid = c.H;
-    g.Y = xp;
-    g.row_of = row_of;
-    g.top_k = c.top_k;
-    g.ldy = c.H;
-    g.residual = static_cast<const __nv_bfloat16*>(residual);
-    const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
-    RMOE_TRY(launch_grouped_gemm(EPI_COMBINE, tm_hs, tm_ws2, g, std::min(sms, tiles), s));
-  } else {
-    RMOE_TRY(launch_combine_rows(xp, row_of, c.T, c.H, c.top_k,
-                                 static_cast<const __nv_bfloat16*>(residual),
-                                 static_cast<__nv_bfloat16*>(out), s));
-  }
+  const void* residual = opts ? opts->residual : nullptr;
+  RMOE_TRY(launch_combine_slots(Y, row_of, c.top_k, c.T, c.H, slots, residual, out, s));
   RMOE_TRY(record(MOE_NUM_STAGES));
   return MOE_OK;
 }

@@ -9,8 +9,9 @@
 //   B  [groups, N, K] bf16 (one weight matrix per group, K-major),
 // differing only in the epilogue:
 //   EPI_SWIGLU   out[r, n] = bf16( silu(D[r, n]) * D[r, I + n] )   (gate|up)
-//   EPI_ROWSCALE out[r, n] = bf16( row_scale[r] * D[r, n] )        (router weight)
-//   EPI_COMBINE  out[t, n] = bf16( sum_j Y[row_of[t,j], n] + D[t, n] [+ res[t, n]] )
+//   EPI_ROWSCALE out[pos[r], n] = bf16( row_scale[r] * D[r, n] )   (router weight;
+//                pos[r] = token-major slot t*(k+1)+j of row r, so that the
+//                combine reads each token's slots contiguously)
 //
 // Kernel shape: persistent, one CTA per SM (192 KB of operand stages), tiles
 // of 128 rows x 256 accumulator columns, K in steps of 64 (one 128-byte
@@ -18,8 +19,9 @@
 //   warp 0      one thread issues TMA tile loads into a 4-stage smem ring;
 //   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators)
 //               and one thread issues tcgen05.mma (M=128, N=256, K=16);
-//   warps 2..5  epilogue: tcgen05.ld the accumulator (warp w reads TMEM
-//               lanes 32*(w%4)..), apply the epilogue, store to global.
+//   warps 2..9  epilogue: tcgen05.ld the accumulator (warp w reads TMEM
+//               lanes 32*(w%4).., columns of half (w-2)/4), apply the
+//               epilogue, store to global.
 // The epilogue of tile i overlaps the MMAs of tile i+1 (double-buffered
 // accumulators).  Every wait is bounded (common.cuh): on a timeout the CTA
 // records MOE_ERR_DEVICE_TIMEOUT, drains its TMA loads and MMAs, frees TMEM
@@ -42,7 +44,8 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;  // producer warp, MMA warp, 8 epilogue warps
+constexpr int EPI_THREADS = 256;
 constexpr int MAX_GROUPS = 128;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
@@ -104,15 +107,18 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const GemmArgs& a, con
 
 __device__ __forceinline__ float silu_f(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
 
+// One epilogue thread owns accumulator row r_in_tile and half `half` of the
+// tile's columns (two warps per TMEM lane quarter).
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tbase,
-                                              const TileCoord& tc, int r_in_tile) {
+                                              const TileCoord& tc, int r_in_tile, int half) {
   const bool valid = r_in_tile < tc.rows;
   const int row = tc.row0 + r_in_tile;
   if constexpr (EPI == EPI_SWIGLU) {
+    // accumulator columns [0,128) gate, [128,256) up; output columns nt*128 + [0,128)
     const int col0 = tc.nt * (BN / 2);
 #pragma unroll 1
-    for (int c = 0; c < BN / 2; c += 32) {
+    for (int c = half * 64; c < half * 64 + 64; c += 32) {
       uint32_t g[32], u[32];
       tmem_ld_32x32b_x32(tbase + c, g);
       tmem_ld_32x32b_x32(tbase + BN / 2 + c, u);
@@ -131,11 +137,12 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tbase,
           dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
       }
     }
-  } else if constexpr (EPI == EPI_ROWSCALE) {
+  } else {  // EPI_ROWSCALE: weighted rows scattered to their token-major slot
     const int col0 = tc.nt * BN;
-    const float w = valid ? a.row_scale[row] : 0.f;
+    const float w = !valid ? 0.f : (a.row_scale ? a.row_scale[row] : 1.0f);
+    const int drow = !valid ? 0 : (a.dest_pos ? a.dest_pos[row] : row * a.dest_mul + a.dest_add);
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = half * 128; c < half * 128 + 128; c += 32) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tbase + c, v);
       tmem_ld_wait();
@@ -144,58 +151,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tbase,
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           pk[i] = pack_bf16x2(w * __uint_as_float(v[2 * i]), w * __uint_as_float(v[2 * i + 1]));
-        uint4* dst = reinterpret_cast<uint4*>(a.out + (size_t)row * a.ldo + col0 + c);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-      }
-    }
-  } else {  // EPI_COMBINE: rows are tokens
-    const int col0 = tc.nt * BN;
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tbase + c, v);
-      tmem_ld_wait();
-      if (valid && col0 + c < a.n_valid) {
-        float s[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] = 0.f;
-        for (int j = 0; j < a.top_k; ++j) {
-          const int r = a.row_of[(size_t)row * a.top_k + j];
-          if (r < 0) continue;
-          const uint4* src = reinterpret_cast<const uint4*>(a.Y + (size_t)r * a.ldy + col0 + c);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 y = src[q];
-            const uint32_t yy[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              s[8 * q + 2 * i] += bf16_lo(yy[i]);
-              s[8 * q + 2 * i + 1] += bf16_hi(yy[i]);
-            }
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] += __uint_as_float(v[i]);
-        if (a.residual) {
-          const uint4* src =
-              reinterpret_cast<const uint4*>(a.residual + (size_t)row * a.ldo + col0 + c);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 y = src[q];
-            const uint32_t yy[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              s[8 * q + 2 * i] += bf16_lo(yy[i]);
-              s[8 * q + 2 * i + 1] += bf16_hi(yy[i]);
-            }
-          }
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
-        uint4* dst = reinterpret_cast<uint4*>(a.out + (size_t)row * a.ldo + col0 + c);
+        uint4* dst = reinterpret_cast<uint4*>(a.out + (size_t)drow * a.ldo + col0 + c);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
@@ -227,7 +183,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&st.tfull[b], 1);
-      mbar_init(&st.tempty[b], 128);
+      mbar_init(&st.tempty[b], EPI_THREADS);
     }
     mbar_init(&st.drain, 1);
     st.abort_flag = 0;
@@ -285,8 +241,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (!ok) {  // let every load in flight land before the CTA can exit
         for (int s = 0; s < STAGES; ++s)
-          if ((armed >> s) & 1u) mbar_wait_drain(&st.full[s], (armed_parity >> s) & 1u,
-                                                 args.timeout_ns);
+          if ((armed >> s) & 1u)
+            mbar_wait_drain(&st.full[s], (armed_parity >> s) & 1u, args.timeout_ns);
       }
     }
   } else if (warp == 1) {
@@ -329,8 +285,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_wait_drain(&st.drain, 0, args.timeout_ns);
     }
   } else {
-    // ------------------------------------------------ epilogue warps 2..5
-    const int q = warp & 3;
+    // ------------------------------------------------ epilogue warps 2..9
+    const int q = warp & 3;           // TMEM lane quarter this warp may read
+    const int half = (warp - 2) >> 2;  // which half of the tile's columns
     const int r_in_tile = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -341,7 +298,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after_sync();
       const uint32_t tbase =
           tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(q * 32) << 16);
-      epilogue_tile<EPI>(args, tbase, tc, r_in_tile);
+      epilogue_tile<EPI>(args, tbase, tc, r_in_tile, half);
       tc_fence_before_sync();
       mbar_arrive(&st.tempty[acc]);
       acc ^= 1;
@@ -420,8 +377,6 @@ cudaError_t launch_grouped_gemm(int epi, const CUtensorMap& tmA, const CUtensorM
       return launch_epi<EPI_SWIGLU>(tmA, tmB, args, grid, stream);
     case EPI_ROWSCALE:
       return launch_epi<EPI_ROWSCALE>(tmA, tmB, args, grid, stream);
-    case EPI_COMBINE:
-      return launch_epi<EPI_COMBINE>(tmA, tmB, args, grid, stream);
     default:
       return cudaErrorInvalidValue;
   }

@@ -12,8 +12,13 @@ struct RouterParams {
   float rsf;
 };
 
+// Router on the tensor cores: scratch holds the 3-term bf16 split of Wr and the
+// fp32 partial logits of the K chunks (router_scratch_bytes).
+int router_splits(int H);
+size_t router_scratch_bytes(int T, int H, int E);
 cudaError_t launch_router(const void* x, const float* Wr, const float* bias, const RouterParams& p,
-                          int32_t* topk_ids, float* topk_w, cudaStream_t stream);
+                          int32_t* topk_ids, float* topk_w, void* scratch, int* status,
+                          unsigned long long timeout_ns, cudaStream_t stream);
 
 // ------------------------------------------------------------------ permute
 constexpr int PERMUTE_TOK = 256;  // tokens per counting block
@@ -26,6 +31,8 @@ struct PermuteOut {
   int* mtile_start;     // [E+1] prefix of ceil(count/MTILE), may be null
   int* row_of;          // [T*k]
   int* tok_of;          // [T*k]
+  int* pos_of = nullptr;  // [T*k] or null: slot position t*slot_stride + j of each row
+  int slot_stride = 0;    // slots per token in the token-major output buffer
   float* w_of;          // [T*k] or null
   void* xp;             // [T*k, H] bf16 or null
 };
@@ -34,7 +41,7 @@ cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const v
                            int H, int E, int top_k, const PermuteOut& o, cudaStream_t stream);
 
 // ------------------------------------------------------------------ grouped GEMM
-enum EpiKind { EPI_SWIGLU = 0, EPI_ROWSCALE = 1, EPI_COMBINE = 2 };
+enum EpiKind { EPI_SWIGLU = 0, EPI_ROWSCALE = 1 };
 
 struct GemmArgs {
   // schedule: groups (experts) of rows, each cut into MTILE-row tiles
@@ -50,12 +57,9 @@ struct GemmArgs {
   __nv_bfloat16* out;      // [rows, ldo]
   int ldo;
   int n_valid;             // valid output columns (N tail mask)
-  const float* row_scale;  // EPI_ROWSCALE: weight of each row
-  const __nv_bfloat16* Y;  // EPI_COMBINE: weighted expert outputs [T*k, ldy]
-  const int* row_of;       // EPI_COMBINE: [T*k]
-  int top_k;
-  int ldy;
-  const __nv_bfloat16* residual;  // EPI_COMBINE: [T, ldo] or null
+  const float* row_scale;  // EPI_ROWSCALE: weight of each row, or null for 1
+  const int* dest_pos;     // EPI_ROWSCALE: output row of each row, or null for
+  int dest_mul, dest_add;  //   row * dest_mul + dest_add
   int* status;
   unsigned long long timeout_ns;
 };
@@ -74,8 +78,10 @@ int num_sms();
 // ------------------------------------------------------------------ misc
 cudaError_t launch_rmsnorm(const void* x, const float* gamma, float eps, int T, int H, void* xn,
                            cudaStream_t stream);
-cudaError_t launch_combine_rows(const void* Y, const int* row_of, int T, int H, int top_k,
-                                const void* residual, void* out, cudaStream_t stream);
+// out[t] = bf16( sum_{j<slots} Y[t*slots + j] [+ residual[t]] ), fp32 sum in slot order;
+// routed slot j < top_k is skipped when row_of[t*top_k + j] < 0 (a rejected expert id).
+cudaError_t launch_combine_slots(const void* Y, const int* row_of, int top_k, int T, int H,
+                                 int slots, const void* residual, void* out, cudaStream_t stream);
 cudaError_t launch_status_reset(int* status, cudaStream_t stream);
 cudaError_t launch_selftest_wait(int* status, unsigned long long timeout_ns, cudaStream_t stream);
 

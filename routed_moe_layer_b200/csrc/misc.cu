@@ -1,6 +1,6 @@
 // Small kernels around the block: RMSNorm for a residual stack (xxqk.cn
 // vLLM-Omni article, "MoE 实现的源码级要点": RMSNorm accumulates in fp32),
-// the restore without a shared expert, and the bounded-wait self test.
+// the restore of the weighted expert slots, and the bounded-wait self test.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -48,42 +48,56 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Restore without a shared expert: out[t] = bf16(sum_j Y[row_of[t,j]] [+ residual[t]]),
-// one warp per token, slots summed in order j = 0..top_k-1.
+// Restore (xxqk.cn vLLM-Omni article, "_restore_tokens": fp32 weighted sum of
+// the expert outputs): the weighted slot rows of token t sit contiguously at
+// Y[t*slots .. t*slots + slots-1] (routed slots, then the shared expert), so
+// one warp per token streams them with 512-byte coalesced loads and sums them
+// in fp32 in slot order, then adds the residual, then rounds once.
 __global__ void __launch_bounds__(256)
-    combine_rows_kernel(const __nv_bfloat16* __restrict__ Y, const int* __restrict__ row_of,
-                        int T, int H, int top_k, const __nv_bfloat16* __restrict__ residual,
-                        __nv_bfloat16* __restrict__ out) {
+    combine_slots_kernel(const __nv_bfloat16* __restrict__ Y, const int* __restrict__ row_of,
+                         int top_k, int T, int H, int slots,
+                         const __nv_bfloat16* __restrict__ residual,
+                         __nv_bfloat16* __restrict__ out) {
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
-  for (int c = lane; c < H / 8; c += 32) {
-    float s[8];
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+    uint32_t skip = 0;  // routed slots of rejected expert ids
+    for (int j = 0; j < top_k; ++j)
+      if (row_of[(size_t)t * top_k + j] < 0) skip |= 1u << j;
+    const uint4* src = reinterpret_cast<const uint4*>(Y + (size_t)t * slots * H);
+    const int hv = H / 8;  // 16-byte vectors per row
+    for (int c = lane; c < hv; c += 32) {
+      float s[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) s[i] = 0.f;
-    for (int j = 0; j < top_k; ++j) {
-      const int r = row_of[(size_t)t * top_k + j];
-      if (r < 0) continue;
-      const uint4 v = reinterpret_cast<const uint4*>(Y + (size_t)r * H)[c];
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      for (int i = 0; i < 8; ++i) s[i] = 0.f;
+      uint4 y[17];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        s[2 * i] += bf16_lo(w[i]);
-        s[2 * i + 1] += bf16_hi(w[i]);
+      for (int j = 0; j < 17; ++j)
+        if (j < slots) y[j] = ((skip >> j) & 1u) ? make_uint4(0, 0, 0, 0) : src[(size_t)j * hv + c];
+#pragma unroll
+      for (int j = 0; j < 17; ++j) {
+        if (j < slots) {
+          const uint32_t w[4] = {y[j].x, y[j].y, y[j].z, y[j].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            s[2 * i] += bf16_lo(w[i]);
+            s[2 * i + 1] += bf16_hi(w[i]);
+          }
+        }
       }
-    }
-    if (residual) {
-      const uint4 v = reinterpret_cast<const uint4*>(residual + (size_t)t * H)[c];
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      if (residual) {
+        const uint4 v = reinterpret_cast<const uint4*>(residual + (size_t)t * H)[c];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        s[2 * i] += bf16_lo(w[i]);
-        s[2 * i + 1] += bf16_hi(w[i]);
+        for (int i = 0; i < 4; ++i) {
+          s[2 * i] += bf16_lo(w[i]);
+          s[2 * i + 1] += bf16_hi(w[i]);
+        }
       }
+      reinterpret_cast<uint4*>(out + (size_t)t * H)[c] =
+          make_uint4(pack_bf16x2(s[0], s[1]), pack_bf16x2(s[2], s[3]), pack_bf16x2(s[4], s[5]),
+                     pack_bf16x2(s[6], s[7]));
     }
-    reinterpret_cast<uint4*>(out + (size_t)t * H)[c] =
-        make_uint4(pack_bf16x2(s[0], s[1]), pack_bf16x2(s[2], s[3]), pack_bf16x2(s[4], s[5]),
-                   pack_bf16x2(s[6], s[7]));
   }
 }
 
@@ -112,11 +126,13 @@ cudaError_t launch_rmsnorm(const void* x, const float* gamma, float eps, int T, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine_rows(const void* Y, const int* row_of, int T, int H, int top_k,
-                                const void* residual, void* out, cudaStream_t stream) {
-  const int grid = (T + 7) / 8;
-  combine_rows_kernel<<<grid, 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(Y), row_of, T, H, top_k,
+cudaError_t launch_combine_slots(const void* Y, const int* row_of, int top_k, int T, int H,
+                                 int slots, const void* residual, void* out, cudaStream_t stream) {
+  int grid = (T + 7) / 8;
+  const int cap = num_sms() * 8;
+  if (grid > cap) grid = cap;
+  combine_slots_kernel<<<grid, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(Y), row_of, top_k, T, H, slots,
       static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(out));
   return cudaGetLastError();
 }

@@ -9,7 +9,8 @@
 //               block histogram = popcounts of the masks.
 //   2. scan:    one CTA turns the block histograms into per-block row bases
 //               and per-expert offsets (+ the prefix of 128-row GEMM tiles).
-//   3. scatter: rank inside the warp = popcount of the lower lanes' bits.
+//   3. scatter: rank inside the warp = popcount of the lower lanes' bits;
+//               also the token-major slot position of every row.
 //   4. gather:  xp[row] = x[tok_of[row]] (skipped when x is not given).
 #include "common.cuh"
 #include "kernels.h"
@@ -139,7 +140,8 @@ __global__ void __launch_bounds__(PT)
     permute_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w,
                            int T, int E, int top_k, const int* __restrict__ blk_base,
                            int* __restrict__ row_of, int* __restrict__ tok_of,
-                           float* __restrict__ w_of, int* status) {
+                           float* __restrict__ w_of, int* __restrict__ pos_of, int slot_stride,
+                           int* status) {
   __shared__ uint32_t masks[PW][MAXE];
   __shared__ int wbase[PW][MAXE];
   build_masks(ids, T, E, top_k, masks, status);
@@ -167,6 +169,7 @@ __global__ void __launch_bounds__(PT)
     row_of[tj] = row;
     tok_of[row] = t;
     if (w_of) w_of[row] = topk_w ? topk_w[tj] : 1.0f;
+    if (pos_of) pos_of[row] = t * slot_stride + j;
   }
 }
 
@@ -197,7 +200,8 @@ cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const v
   permute_scan_kernel<<<1, 1024, 0, stream>>>(o.blk_hist, nblk, E, o.expert_offsets,
                                               o.mtile_start);
   permute_scatter_kernel<<<nblk, PT, 0, stream>>>(topk_ids, topk_w, T, E, top_k, o.blk_hist,
-                                                  o.row_of, o.tok_of, o.w_of, o.status);
+                                                  o.row_of, o.tok_of, o.w_of, o.pos_of,
+                                                  o.slot_stride, o.status);
   if (o.xp && x) {
     const int R = T * top_k;
     int grid = (R + 7) / 8;

@@ -4,10 +4,21 @@
 // "MoE 实现的源码级要点": selection on bias-corrected scores, gating weights
 // from the raw scores, norm_topk_prob renormalisation).
 //
-// One CTA scores ROUTER_TOK tokens against all experts with fp32 FMAs (x is
-// exactly representable in fp32, so each logit is an fp32 dot product of the
-// bf16 token and the fp32 router row), parks the logits in shared memory,
-// then one warp per token does the three selections with warp shuffles.
+// fp32-faithful logits on the bf16 tensor cores.  Every fp32 router weight is
+// the exact sum of three bf16 terms (hi = bf16(w), mid = bf16(w - hi),
+// lo = w - hi - mid: each residual has at most 16, then 8 significant bits).
+// Tokens are bf16, so each product token x term is exact in fp32 and
+// logits = x.hi^T + x.mid^T + x.lo^T accumulate in fp32 in TMEM -- an fp32 dot
+// product of the bf16 token and the fp32 router row, up to summation order.
+//   1. router_split_kernel    Wr [E,H] fp32 -> Wr3 [3,E,H] bf16
+//   2. router_gemm_kernel     tcgen05 128 tokens x 128 experts tiles, K split
+//                             into a number of chunks that depends on H only
+//                             (so a token's logits never depend on T); each
+//                             chunk's fp32 partial goes to [S,T,E]
+//   3. router_select_kernel   one warp per token: sums the S partials in order,
+//                             then sigmoid, bias, group top-2 sums, group
+//                             selection, expert selection and weights with
+//                             warp shuffles.
 #include <float.h>
 #include <limits.h>
 
@@ -18,20 +29,181 @@ namespace rmoe {
 
 namespace {
 
-constexpr int ROUTER_TOK = 64;   // tokens per CTA
-constexpr int ROUTER_EP = 128;   // expert slots per CTA (E <= 128)
-constexpr int ROUTER_KC = 32;    // K chunk
-constexpr int ROUTER_THREADS = 256;
-constexpr int XS_LD = ROUTER_TOK + 4;
-constexpr int WS_LD = ROUTER_EP + 4;
-constexpr int LG_LD = ROUTER_EP + 1;
 constexpr unsigned FULL = 0xffffffffu;
+constexpr int RBM = 128;  // tokens per tile
+constexpr int RBN = 128;  // experts per tile (E <= 128)
+constexpr int RBK = 64;
+constexpr int RSTAGES = 3;
+constexpr int R_A_BYTES = RBM * RBK * 2;
+constexpr int R_B_BYTES = RBN * RBK * 2;
+constexpr int R_STAGE_BYTES = R_A_BYTES + 3 * R_B_BYTES;
+constexpr int R_THREADS = 192;
+constexpr uint32_t R_TMEM_COLS = 128;
+constexpr uint32_t R_IDESC = idesc_bf16_f32(RBM, RBN);
 
-struct RouterSmem {
-  float xs[ROUTER_KC][XS_LD];
-  float ws[ROUTER_KC][WS_LD];
-  float logits[ROUTER_TOK][LG_LD];
+struct __align__(8) RouterTail {
+  uint64_t full[RSTAGES];
+  uint64_t empty[RSTAGES];
+  uint64_t tfull;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
 };
+
+constexpr size_t R_SMEM_BYTES = 1024 + (size_t)RSTAGES * R_STAGE_BYTES + sizeof(RouterTail);
+
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > timeout_ns) return;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    router_split_kernel(const float* __restrict__ Wr, size_t n, __nv_bfloat16* __restrict__ Wr3) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float w = Wr[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);  // exact
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);  // exact, fits in bf16
+    Wr3[i] = hi;
+    Wr3[n + i] = mid;
+    Wr3[2 * n + i] = __float2bfloat16_rn(r2);
+  }
+}
+
+// grid (m_tiles, S): tile blockIdx.x of 128 tokens, K chunk blockIdx.y.
+__global__ void __launch_bounds__(R_THREADS, 1)
+    router_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
+                       const __grid_constant__ CUtensorMap tmW3, int T, int E, int k_steps,
+                       int S, float* __restrict__ partial, int* status,
+                       unsigned long long timeout_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  RouterTail& st = *reinterpret_cast<RouterTail*>(smem + (size_t)RSTAGES * R_STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * RBM;
+  const int s = blockIdx.y;
+  const int kb = (int)((long long)s * k_steps / S), ke = (int)((long long)(s + 1) * k_steps / S);
+  const int nk = ke - kb;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < RSTAGES; ++i) {
+      mbar_init(&st.full[i], 1);
+      mbar_init(&st.empty[i], 1);
+    }
+    mbar_init(&st.tfull, 1);
+    mbar_init(&st.drain, 1);
+    st.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x == 32) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW3);
+  }
+  if (warp == 1) {
+    tmem_alloc(&st.tmem_base, R_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = st.tmem_base;
+  const WaitCtx wc{&st.abort_flag, status, timeout_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int i = 0; i < nk; ++i) {
+        const int stage = i % RSTAGES;
+        const uint32_t phase = (i / RSTAGES) & 1u;
+        if (!mbar_wait(&st.empty[stage], phase ^ 1u, wc, 40)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + (size_t)stage * R_STAGE_BYTES;
+        mbar_arrive_expect_tx(&st.full[stage], R_STAGE_BYTES);
+        const int kc = (kb + i) * RBK;
+        tma_load_2d(sa, &tmX, &st.full[stage], kc, m0);
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+          tma_load_3d(sa + R_A_BYTES + t * R_B_BYTES, &tmW3, &st.full[stage], kc, 0, t);
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+      }
+      if (!ok) {
+        for (int i = 0; i < RSTAGES; ++i)
+          if ((armed >> i) & 1u) wait_drain(&st.full[i], (armed_parity >> i) & 1u, timeout_ns);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = true;
+      for (int i = 0; i < nk; ++i) {
+        const int stage = i % RSTAGES;
+        const uint32_t phase = (i / RSTAGES) & 1u;
+        if (!mbar_wait(&st.full[stage], phase, wc, 41)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t sa = smem_u32(smem + (size_t)stage * R_STAGE_BYTES);
+        const uint64_t da = sdesc_kmajor_sw128(sa);
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+          const uint64_t db = sdesc_kmajor_sw128(sa + R_A_BYTES + t * R_B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < RBK / 16; ++kk)
+            umma_bf16_ss(tmem_base, da + 2 * kk, db + 2 * kk, R_IDESC,
+                         (i | t | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit(&st.empty[stage]);
+      }
+      if (ok) umma_commit(&st.tfull);
+      umma_commit(&st.drain);
+      wait_drain(&st.drain, 0, timeout_ns);
+    }
+  } else {
+    const int q = warp & 3;
+    const bool ok = mbar_wait(&st.tfull, 0, wc, 42);
+    if (__all_sync(FULL, ok)) {
+      tc_fence_after_sync();
+      const int row = m0 + q * 32 + lane;
+      float* dst = partial + ((size_t)s * T + row) * E;
+#pragma unroll 1
+      for (int c = 0; c < RBN; c += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + c, v);
+        tmem_ld_wait();
+        if (row < T && c < E) {
+          if (c + 32 <= E && (E & 3) == 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              reinterpret_cast<float4*>(dst + c)[i] =
+                  make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                              __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c + i < E) dst[c + i] = __uint_as_float(v[i]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, R_TMEM_COLS);
+  }
+}
 
 // Warp-wide argmax: larger value wins, equal values go to the lower index.
 __device__ __forceinline__ void warp_argmax(float& v, int& idx) {
@@ -46,135 +218,75 @@ __device__ __forceinline__ void warp_argmax(float& v, int& idx) {
   }
 }
 
-__global__ void __launch_bounds__(ROUTER_THREADS)
-    router_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ Wr,
-                  const float* __restrict__ bias, RouterParams p, int32_t* __restrict__ topk_ids,
-                  float* __restrict__ topk_w) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  RouterSmem& sm = *reinterpret_cast<RouterSmem*>(smem_raw);
-  const int tid = threadIdx.x;
-  const int tok0 = blockIdx.x * ROUTER_TOK;
-  const int T = p.T, H = p.H, E = p.E;
+// One warp per token; lane l holds experts l + 32*i.
+constexpr int SEL_WARPS = 8;
 
-  // ---------------------------------------------------------------- logits
-  const int tx = tid & 15;  // experts tx*8 .. tx*8+7
-  const int ty = tid >> 4;  // tokens  ty*4 .. ty*4+3
-  float acc[4][8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-
-  for (int k0 = 0; k0 < H; k0 += ROUTER_KC) {
-    {  // x chunk: 64 tokens x 32 k, one 8-element vector per thread
-      const int t = tid >> 2, kq = tid & 3;
-      const int tg = tok0 + t;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (tg < T) v = *reinterpret_cast<const uint4*>(x + (size_t)tg * H + k0 + kq * 8);
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        sm.xs[kq * 8 + 2 * i][t] = bf16_lo(w4[i]);
-        sm.xs[kq * 8 + 2 * i + 1][t] = bf16_hi(w4[i]);
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {  // W chunk: 128 experts x 32 k fp32
-      const int f = tid + r * ROUTER_THREADS;
-      const int e = f >> 3, q = f & 7;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < E) v = *reinterpret_cast<const float4*>(Wr + (size_t)e * H + k0 + q * 4);
-      sm.ws[q * 4 + 0][e] = v.x;
-      sm.ws[q * 4 + 1][e] = v.y;
-      sm.ws[q * 4 + 2][e] = v.z;
-      sm.ws[q * 4 + 3][e] = v.w;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int k = 0; k < ROUTER_KC; ++k) {
-      const float4 a = *reinterpret_cast<const float4*>(&sm.xs[k][ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&sm.ws[k][tx * 8]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&sm.ws[k][tx * 8 + 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) sm.logits[ty * 4 + i][tx * 8 + j] = acc[i][j];
-  __syncthreads();
-
-  // ---------------------------------------------------------------- selection
-  const int warp = tid >> 5, lane = tid & 31;
+__global__ void __launch_bounds__(SEL_WARPS * 32)
+    router_select_kernel(const float* __restrict__ partial, int S, const float* __restrict__ bias,
+                         RouterParams p, int32_t* __restrict__ topk_ids,
+                         float* __restrict__ topk_w) {
+  constexpr int NE = RBN / 32;
+  __shared__ float sc[SEL_WARPS][RBN];  // bias-corrected scores of the warp's token
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int warps = gridDim.x * SEL_WARPS;
+  const int T = p.T, E = p.E;
   const int gs = E / p.n_group;
-  constexpr int NE = ROUTER_EP / 32;  // experts per lane: e = lane + 32*i
+  const bool group_step = p.topk_group < p.n_group;
   float b[NE];
+  int grp[NE];  // group of each held expert (computed once)
 #pragma unroll
   for (int i = 0; i < NE; ++i) {
     const int e = lane + 32 * i;
     b[i] = (e < E) ? bias[e] : 0.f;
+    grp[i] = (e < E) ? e / gs : 0;
   }
-  for (int tl = warp; tl < ROUTER_TOK; tl += ROUTER_THREADS / 32) {
-    const int t = tok0 + tl;
-    if (t >= T) break;  // warp-uniform
+  for (int t = blockIdx.x * SEL_WARPS + wib; t < T; t += warps) {
     float s[NE], c[NE];
     bool avail[NE];
 #pragma unroll
     for (int i = 0; i < NE; ++i) {
       const int e = lane + 32 * i;
-      const float l = sm.logits[tl][e < ROUTER_EP ? e : 0];
+      avail[i] = e < E;
+      float l = 0.f;
+      if (avail[i]) {
+        l = partial[(size_t)t * E + e];
+        for (int k = 1; k < S; ++k) l += partial[((size_t)k * T + t) * E + e];
+      }
       s[i] = 1.0f / (1.0f + expf(-l));
       c[i] = s[i] + b[i];
-      avail[i] = e < E;
     }
-    // group-limited candidates
-    if (p.topk_group < p.n_group) {
-      uint32_t kept = 0;
-      float G[32];
-      for (int j = 0; j < p.n_group; ++j) {
+    if (group_step) {
+#pragma unroll
+      for (int i = 0; i < NE; ++i)
+        if (avail[i]) sc[wib][lane + 32 * i] = c[i];
+      __syncwarp();
+      // lane j < n_group: group score = sum of the two largest c of group j
+      float G = -FLT_MAX;
+      if (lane < p.n_group) {
         float v1 = -FLT_MAX, v2 = -FLT_MAX;
-        int i1 = INT_MAX;
-#pragma unroll
-        for (int i = 0; i < NE; ++i) {
-          const int e = lane + 32 * i;
-          if (avail[i] && e / gs == j && (c[i] > v1 || (c[i] == v1 && e < i1))) {
-            v1 = c[i];
-            i1 = e;
+        const float* g = &sc[wib][lane * gs];
+        for (int q = 0; q < gs; ++q) {
+          const float v = g[q];
+          if (v > v1) {
+            v2 = v1;
+            v1 = v;
+          } else if (v > v2) {
+            v2 = v;
           }
         }
-        warp_argmax(v1, i1);
-        // second best of the group: best excluding i1
+        G = v1 + v2;
+      }
+      // rank of each group: larger score first, ties to the lower group index
+      int rank = 0;
+      for (int m = 0; m < p.n_group; ++m) {
+        const float Gm = __shfl_sync(FULL, G, m);
+        if (Gm > G || (Gm == G && m < lane)) ++rank;
+      }
+      const uint32_t kept = __ballot_sync(FULL, lane < p.n_group && rank < p.topk_group);
 #pragma unroll
-        for (int i = 0; i < NE; ++i) {
-          const int e = lane + 32 * i;
-          if (avail[i] && e / gs == j && e != i1 && c[i] > v2) v2 = c[i];
-        }
-        int i2 = 0;
-        warp_argmax(v2, i2);
-        G[j] = v1 + v2;
-      }
-      for (int r = 0; r < p.topk_group; ++r) {
-        int bj = -1;
-        float bv = -FLT_MAX;
-        for (int j = 0; j < p.n_group; ++j) {
-          if (!((kept >> j) & 1u) && (bj < 0 || G[j] > bv)) {
-            bv = G[j];
-            bj = j;
-          }
-        }
-        kept |= 1u << bj;
-      }
-#pragma unroll
-      for (int i = 0; i < NE; ++i) {
-        const int e = lane + 32 * i;
-        if (avail[i] && !((kept >> (e / gs)) & 1u)) avail[i] = false;
-      }
+      for (int i = 0; i < NE; ++i)
+        if (avail[i] && !((kept >> grp[i]) & 1u)) avail[i] = false;
+      __syncwarp();
     }
     // top_k experts among the candidates
     int my_id = -1;
@@ -205,7 +317,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS)
         }
       } else {
         sv = 0.f;
-        idx = -1;  // no candidate left (non-finite scores); permute reports it
+        idx = -1;  // no candidate left (non-finite scores); the permutation reports it
       }
       sum += sv;
       if (lane == r) {
@@ -223,15 +335,43 @@ __global__ void __launch_bounds__(ROUTER_THREADS)
 
 }  // namespace
 
+int router_splits(int H) {
+  const int k_steps = H / RBK;
+  return k_steps / 8 > 1 ? k_steps / 8 : 1;
+}
+
+size_t router_scratch_bytes(int T, int H, int E) {
+  const size_t a = ((size_t)3 * E * H * 2 + 255) & ~(size_t)255;
+  return a + (size_t)router_splits(H) * T * E * 4;
+}
+
 cudaError_t launch_router(const void* x, const float* Wr, const float* bias, const RouterParams& p,
-                          int32_t* topk_ids, float* topk_w, cudaStream_t stream) {
-  const int grid = (p.T + ROUTER_TOK - 1) / ROUTER_TOK;
-  const size_t smem = sizeof(RouterSmem);
-  cudaError_t err =
-      cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                          int32_t* topk_ids, float* topk_w, void* scratch, int* status,
+                          unsigned long long timeout_ns, cudaStream_t stream) {
+  const int T = p.T, H = p.H, E = p.E;
+  __nv_bfloat16* Wr3 = static_cast<__nv_bfloat16*>(scratch);
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) +
+                                            (((size_t)3 * E * H * 2 + 255) & ~(size_t)255));
+  const size_t n = (size_t)E * H;
+  router_split_kernel<<<(int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, stream>>>(
+      Wr, n, Wr3);
+  CUtensorMap tmX, tmW3;
+  cudaError_t err = make_tmap_2d(&tmX, x, (uint64_t)T, (uint64_t)H);
   if (err != cudaSuccess) return err;
-  router_kernel<<<grid, ROUTER_THREADS, smem, stream>>>(
-      static_cast<const __nv_bfloat16*>(x), Wr, bias, p, topk_ids, topk_w);
+  err = make_tmap_3d(&tmW3, Wr3, 3, (uint64_t)E, (uint64_t)H);
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)R_SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  const int S = router_splits(H);
+  const dim3 grid((T + RBM - 1) / RBM, S);
+  router_gemm_kernel<<<grid, R_THREADS, R_SMEM_BYTES, stream>>>(tmX, tmW3, T, E, H / RBK, S,
+                                                                 partial, status, timeout_ns);
+  int sel_grid = (T + SEL_WARPS - 1) / SEL_WARPS;
+  const int cap = num_sms() * 16;
+  if (sel_grid > cap) sel_grid = cap;
+  router_select_kernel<<<sel_grid, SEL_WARPS * 32, 0, stream>>>(partial, S, bias, p, topk_ids,
+                                                                 topk_w);
   return cudaGetLastError();
 }
 

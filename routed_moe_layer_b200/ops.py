@@ -24,7 +24,7 @@ STATUS_NAMES = {
     3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT",
     6: "MOE_ERR_DEVICE_INDEX", 7: "MOE_ERR_NO_DEVICE",
 }
-STAGES = ("router", "permute", "expert_up", "expert_down", "shared_up", "combine")
+STAGES = ("router", "permute", "expert_up", "expert_down", "shared_expert", "combine")
 NUM_STAGES = len(STAGES)
 
 
@@ -165,8 +165,9 @@ def route(x: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor, cfg: BlockConfi
     ids = torch.empty((T, cfg.top_k), dtype=torch.int32, device=x.device)
     w = torch.empty((T, cfg.top_k), dtype=torch.float32, device=x.device)
     c = cfg.c()
+    ws = alloc_workspace(lib().moe_route_workspace_bytes(ctypes.byref(c)), x.device)
     _check(lib().moe_route(_ptr(x), _ptr(Wr), _ptr(bias), ctypes.byref(c), _ptr(ids), _ptr(w),
-                           None, 0, _stream_ptr()), "moe_route")
+                           _ptr(ws), ws.numel(), _stream_ptr()), "moe_route")
     return ids, w
 
 
