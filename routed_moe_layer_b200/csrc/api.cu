@@ -275,7 +275,9 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
   o.xp = xp;
   RMOE_TRY(launch_permute(ids, tw, x, c.T, c.H, c.E, c.top_k, o, s));
 
-  const int mt_bound = (int)(R / MTILE) + c.E;  // every expert adds at most one partial tile
+  // tiles of MTILE rows, each computed by a pair of CTAs; every expert adds at
+  // most one partial tile
+  const int mt_bound = (int)(R / MTILE) + c.E;
   GemmArgs a;
   memset(&a, 0, sizeof(a));
   a.status = status;
@@ -294,7 +296,7 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
     g.out = h;
     g.ldo = c.I;
     g.n_valid = c.I;
-    const int grid = (int)std::min<long long>(sms, (long long)mt_bound * g.n_tiles);
+    const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
     RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_xp, tm_w13, g, grid, s));
   }
   RMOE_TRY(record(MOE_STAGE_EXPERT_DOWN));
@@ -312,7 +314,7 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
     g.n_valid = c.H;
     g.row_scale = o.w_of;
     g.dest_pos = o.pos_of;
-    const int grid = (int)std::min<long long>(sms, (long long)mt_bound * g.n_tiles);
+    const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
     RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, g, grid, s));
   }
   RMOE_TRY(record(MOE_STAGE_SHARED_EXPERT));
@@ -328,7 +330,7 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
       g.ldo = c.I_shared;
       g.n_valid = c.I_shared;
       const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
-      RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_x, tm_ws13, g, std::min(sms, tiles), s));
+      RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_x, tm_ws13, g, std::min(sms, 2 * tiles), s));
     }
     {  // Y[t*slots + top_k] = hs . Ws2^T  (unscaled)
       GemmArgs g = a;
@@ -343,7 +345,7 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
       g.dest_mul = slots;
       g.dest_add = c.top_k;
       const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
-      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_hs, tm_ws2, g, std::min(sms, tiles), s));
+      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_hs, tm_ws2, g, std::min(sms, 2 * tiles), s));
     }
   }
   RMOE_TRY(record(MOE_STAGE_COMBINE));

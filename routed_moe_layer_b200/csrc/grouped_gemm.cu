@@ -13,15 +13,21 @@
 //                pos[r] = token-major slot t*(k+1)+j of row r, so that the
 //                combine reads each token's slots contiguously)
 //
-// Kernel shape: persistent, one CTA per SM (192 KB of operand stages), tiles
-// of 128 rows x 256 accumulator columns, K in steps of 64 (one 128-byte
-// swizzle atom).  Warp roles:
-//   warp 0      one thread issues TMA tile loads into a 4-stage smem ring;
-//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators)
-//               and one thread issues tcgen05.mma (M=128, N=256, K=16);
-//   warps 2..9  epilogue: tcgen05.ld the accumulator (warp w reads TMEM
-//               lanes 32*(w%4).., columns of half (w-2)/4), apply the
-//               epilogue, store to global.
+// Kernel shape: persistent clusters of two CTAs on neighbouring SMs sharing
+// one tcgen05 pair MMA (cta_group::2, M=256, N=256, K=16): a tile is 256 rows
+// (128 in each CTA) x 256 accumulator columns; each CTA loads its own 128 A
+// rows and its half (128 rows) of the B tile per 64-wide K step into a
+// 6-stage shared-memory ring, so each SM moves 32 KB per step instead of 48.
+// Warp roles (both CTAs):
+//   warp 0      one thread issues TMA tile loads; their bytes are counted on
+//               the leader CTA's barrier;
+//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulator
+//               halves); in the leader one thread issues the pair MMAs and
+//               commits to both CTAs' barriers;
+//   warps 2..9  epilogue: tcgen05.ld the CTA's accumulator half (warp w
+//               reads TMEM lanes 32*(w%4).., columns of half (w-2)/4), apply
+//               the epilogue, store to global; then release the accumulator
+//               on the leader's barrier.
 // The epilogue of tile i overlaps the MMAs of tile i+1 (double-buffered
 // accumulators).  Every wait is bounded (common.cuh): on a timeout the CTA
 // records MOE_ERR_DEVICE_TIMEOUT, drains its TMA loads and MMAs, frees TMEM
@@ -37,18 +43,20 @@ namespace rmoe {
 
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;           // rows per CTA
+constexpr int TILE_M = 2 * BM;    // rows per pair tile
+constexpr int BN = 256;           // accumulator columns
 constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BK * 2;        // this CTA's A rows
+constexpr int B_BYTES = (BN / 2) * BK * 2;  // this CTA's half of the B tile
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 320;  // producer warp, MMA warp, 8 epilogue warps
 constexpr int EPI_THREADS = 256;
 constexpr int MAX_GROUPS = 128;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN);
+constexpr int EPI_WARPS = EPI_THREADS / 32;
 constexpr unsigned FULL = 0xffffffffu;
 
 struct __align__(8) SmemTail {
@@ -87,8 +95,8 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const GemmArgs& a, con
   c.nt = tile - mt * a.n_tiles;
   if (a.mtile_start == nullptr) {
     c.g = 0;
-    c.row0 = mt * BM;
-    c.rows = min(BM, a.single_rows - c.row0);
+    c.row0 = mt * TILE_M;
+    c.rows = min(TILE_M, a.single_rows - c.row0);
     return c;
   }
   int lo = 0, hi = a.num_groups;  // largest g with mts[g] <= mt
@@ -100,18 +108,47 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const GemmArgs& a, con
       hi = mid;
   }
   c.g = lo;
-  c.row0 = rs[lo] + (mt - mts[lo]) * BM;
-  c.rows = min(BM, rs[lo + 1] - c.row0);
+  c.row0 = rs[lo] + (mt - mts[lo]) * TILE_M;
+  c.rows = min(TILE_M, rs[lo + 1] - c.row0);
+  return c;
+}
+
+// The part of a pair tile that CTA `rank` holds: rows [row0 + 128*rank, +128).
+__device__ __forceinline__ TileCoord cta_part(TileCoord c, uint32_t rank) {
+  c.row0 += BM * (int)rank;
+  c.rows = max(0, min(BM, c.rows - BM * (int)rank));
   return c;
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
 
+// Per-row inputs of the epilogue, read before the accumulator is waited for
+// so that their latency hides behind the MMAs.
+struct RowIn {
+  float w;   // EPI_ROWSCALE: row weight
+  int drow;  // EPI_ROWSCALE: output row
+};
+
+template <int EPI>
+__device__ __forceinline__ RowIn epilogue_row_inputs(const GemmArgs& a, const TileCoord& tc,
+                                                     int r_in_tile) {
+  RowIn in{0.f, 0};
+  if constexpr (EPI == EPI_ROWSCALE) {
+    if (r_in_tile < tc.rows) {
+      const int row = tc.row0 + r_in_tile;
+      in.w = a.row_scale ? a.row_scale[row] : 1.0f;
+      in.drow = a.dest_pos ? a.dest_pos[row] : row * a.dest_mul + a.dest_add;
+    }
+  }
+  return in;
+}
+
 // One epilogue thread owns accumulator row r_in_tile and half `half` of the
 // tile's columns (two warps per TMEM lane quarter).
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tbase,
-                                              const TileCoord& tc, int r_in_tile, int half) {
+                                              const TileCoord& tc, int r_in_tile, int half,
+                                              const RowIn& in) {
   const bool valid = r_in_tile < tc.rows;
   const int row = tc.row0 + r_in_tile;
   if constexpr (EPI == EPI_SWIGLU) {
@@ -139,8 +176,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tbase,
     }
   } else {  // EPI_ROWSCALE: weighted rows scattered to their token-major slot
     const int col0 = tc.nt * BN;
-    const float w = !valid ? 0.f : (a.row_scale ? a.row_scale[row] : 1.0f);
-    const int drow = !valid ? 0 : (a.dest_pos ? a.dest_pos[row] : row * a.dest_mul + a.dest_add);
+    const float w = in.w;
+    const int drow = in.drow;
 #pragma unroll 1
     for (int c = half * 128; c < half * 128 + 128; c += 32) {
       uint32_t v[32];
@@ -161,7 +198,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tbase,
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
@@ -169,6 +206,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                                              ~static_cast<uintptr_t>(1023));
   SmemTail& st = *reinterpret_cast<SmemTail*>(smem + (size_t)STAGES * STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: leader (issues the MMAs), 1: peer
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
 
   if (args.mtile_start) {
     for (int i = threadIdx.x; i <= args.num_groups; i += THREADS) {
@@ -178,12 +218,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&st.full[s], 1);
-      mbar_init(&st.empty[s], 1);
+      mbar_init(&st.full[s], 1);   // leader: its producer's expect-tx arrive
+      mbar_init(&st.empty[s], 1);  // both: one commit from the leader's MMA thread
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&st.tfull[b], 1);
-      mbar_init(&st.tempty[b], EPI_THREADS);
+      mbar_init(&st.tfull[b], 1);                 // both: one commit
+      mbar_init(&st.tempty[b], 2 * EPI_WARPS);    // leader: every epilogue warp of both CTAs
     }
     mbar_init(&st.drain, 1);
     st.abort_flag = 0;
@@ -195,13 +235,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   __syncthreads();
   const int total_m = args.mtile_start ? st.mt_start[args.num_groups]
-                                       : (args.single_rows + BM - 1) / BM;
+                                       : (args.single_rows + TILE_M - 1) / TILE_M;
   const int total = total_m * args.n_tiles;
-  if (static_cast<int>(blockIdx.x) >= total) return;  // CTA-uniform; nothing allocated yet
+  if (cluster >= total) return;  // the same for both CTAs of the cluster; nothing allocated yet
+  cluster_sync();                // both CTAs' barriers exist before any cross-CTA traffic
 
   if (warp == 1) {
-    tmem_alloc(&st.tmem_base, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(&st.tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -211,26 +252,25 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------ TMA producer
+      // ------------------------------------------------ TMA producer (both CTAs)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage bit: armed at least once / last parity
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      for (int tile = cluster; ok && tile < total; tile += nclusters) {
         const TileCoord tc = tile_coord(tile, args, st.mt_start, st.row_start);
-        const int nb0 = tc.nt * args.n_out_tile;
+        const int a_row = tc.row0 + BM * (int)rank;
+        const int b_row = tc.nt * args.n_out_tile + (int)rank * args.b_second;
         for (int ks = 0; ks < args.k_steps; ++ks) {
           if (!mbar_wait(&st.empty[stage], phase ^ 1u, wc, 10)) {
             ok = false;
             break;
           }
           uint8_t* sa = smem + (size_t)stage * STAGE_BYTES;
-          uint8_t* sb = sa + A_BYTES;
-          mbar_arrive_expect_tx(&st.full[stage], STAGE_BYTES);
-          tma_load_2d(sa, &tmA, &st.full[stage], ks * BK, tc.row0);
-          tma_load_3d(sb, &tmB, &st.full[stage], ks * BK, nb0, tc.g);
-          tma_load_3d(sb + B_BYTES / 2, &tmB, &st.full[stage], ks * BK, nb0 + args.b_second,
-                      tc.g);
+          const uint32_t full_leader = mapa_shared(smem_u32(&st.full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&st.full[stage], 2 * STAGE_BYTES);
+          tma_load_2d_pair(sa, &tmA, full_leader, ks * BK, a_row);
+          tma_load_3d_pair(sa + A_BYTES, &tmB, full_leader, ks * BK, b_row, tc.g);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -239,21 +279,21 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      if (!ok) {  // let every load in flight land before the CTA can exit
+      if (!ok && leader) {  // both CTAs' loads are counted on the leader's barriers
         for (int s = 0; s < STAGES; ++s)
           if ((armed >> s) & 1u)
             mbar_wait_drain(&st.full[s], (armed_parity >> s) & 1u, args.timeout_ns);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------ MMA issuer
+    if (lane == 0 && leader) {
+      // ------------------------------------------------ pair MMA issuer (leader)
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      for (int tile = cluster; ok && tile < total; tile += nclusters) {
         if (!mbar_wait(&st.tempty[acc], acc_phase ^ 1u, wc, 20)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -268,49 +308,55 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint64_t db = sdesc_kmajor_sw128(sa + A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes along K per UMMA_K=16
-            umma_bf16_ss(d_tmem, da + 2 * kk, db + 2 * kk, IDESC, (ks | kk) != 0 ? 1u : 0u);
-          umma_commit(&st.empty[stage]);
+            umma_bf16_ss_pair(d_tmem, da + 2 * kk, db + 2 * kk, IDESC, (ks | kk) != 0 ? 1u : 0u);
+          umma_commit_pair_mask(&st.empty[stage], 0x3);  // free the stage in both CTAs
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(&st.tfull[acc]);
+        umma_commit_pair_mask(&st.tfull[acc], 0x3);  // accumulator ready in both CTAs
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       // every MMA issued by this thread completes before TMEM is released
-      umma_commit(&st.drain);
+      umma_commit_pair_mask(&st.drain, 0x1);
       mbar_wait_drain(&st.drain, 0, args.timeout_ns);
     }
   } else {
-    // ------------------------------------------------ epilogue warps 2..9
-    const int q = warp & 3;           // TMEM lane quarter this warp may read
+    // ------------------------------------------------ epilogue warps 2..9 (both CTAs)
+    const int q = warp & 3;            // TMEM lane quarter this warp may read
     const int half = (warp - 2) >> 2;  // which half of the tile's columns
     const int r_in_tile = q * 32 + lane;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&st.tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&st.tempty[1]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const TileCoord tc = tile_coord(tile, args, st.mt_start, st.row_start);
+    for (int tile = cluster; tile < total; tile += nclusters) {
+      const TileCoord tc = cta_part(tile_coord(tile, args, st.mt_start, st.row_start), rank);
+      const RowIn in = epilogue_row_inputs<EPI>(args, tc, r_in_tile);
       const bool ok = mbar_wait(&st.tfull[acc], acc_phase, wc, 30);
       if (!__all_sync(FULL, ok)) break;  // warp-uniform exit
       tc_fence_after_sync();
       const uint32_t tbase =
           tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(q * 32) << 16);
-      epilogue_tile<EPI>(args, tbase, tc, r_in_tile, half);
+      epilogue_tile<EPI>(args, tbase, tc, r_in_tile, half, in);
       tc_fence_before_sync();
-      mbar_arrive(&st.tempty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(acc == 0 ? tempty_leader0 : tempty_leader1);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
   }
 
+  // both CTAs are done with both accumulators before either frees TMEM or exits
   tc_fence_before_sync();
   __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -334,6 +380,8 @@ cudaError_t launch_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const Gem
   static cudaError_t attr = cudaFuncSetAttribute(
       grouped_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (attr != cudaSuccess) return attr;
+  grid &= ~1;  // clusters of two CTAs
+  if (grid < 2) grid = 2;
   grouped_gemm_kernel<EPI><<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, args);
   return cudaGetLastError();
 }

@@ -22,7 +22,7 @@ cudaError_t launch_router(const void* x, const float* Wr, const float* bias, con
 
 // ------------------------------------------------------------------ permute
 constexpr int PERMUTE_TOK = 256;  // tokens per counting block
-constexpr int MTILE = 128;        // rows per GEMM tile (the M of one UMMA)
+constexpr int MTILE = 256;        // rows per grouped-GEMM tile (one CTA-pair MMA)
 
 struct PermuteOut {
   int* status;          // DevStatus
@@ -44,7 +44,7 @@ cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const v
 enum EpiKind { EPI_SWIGLU = 0, EPI_ROWSCALE = 1 };
 
 struct GemmArgs {
-  // schedule: groups (experts) of rows, each cut into MTILE-row tiles
+  // schedule: groups (experts) of rows, each cut into MTILE-row tiles (one per CTA pair)
   const int* mtile_start;  // [num_groups+1] device prefix of tiles per group; null: one group
   const int* row_start;    // [num_groups+1] device first row of each group
   int num_groups;

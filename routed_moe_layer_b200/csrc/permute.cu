@@ -11,7 +11,8 @@
 //               and per-expert offsets (+ the prefix of 128-row GEMM tiles).
 //   3. scatter: rank inside the warp = popcount of the lower lanes' bits;
 //               also the token-major slot position of every row.
-//   4. gather:  xp[row] = x[tok_of[row]] (skipped when x is not given).
+//   4. gather:  xp[row] = x[tok_of[row]], walking tokens in order so that each
+//               token row is read once (skipped when x is not given).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -173,21 +174,23 @@ __global__ void __launch_bounds__(PT)
   }
 }
 
-// One warp per destination row; 16-byte vectors.
+// One warp per token: x[t] is read once (512 bytes per warp step) and written
+// to the token's top_k rows; row_of gives them (-1: skipped id).
 __global__ void __launch_bounds__(256)
-    gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int* __restrict__ tok_of,
-                       int R, int H, int T, __nv_bfloat16* __restrict__ xp) {
+    gather_tokens_kernel(const __nv_bfloat16* __restrict__ x, const int* __restrict__ row_of,
+                         int T, int H, int top_k, __nv_bfloat16* __restrict__ xp) {
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (blockDim.x >> 5);
-  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += warps) {
-    const int t = tok_of[r];
-    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * H);
-    if (t < 0 || t >= T) {
-      for (int c = lane; c < H / 8; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
-      continue;
-    }
+  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+    const int my_row = lane < top_k ? row_of[(size_t)t * top_k + lane] : -1;
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
-    for (int c = lane; c < H / 8; c += 32) dst[c] = src[c];
+    for (int c = lane; c < H / 8; c += 32) {
+      const uint4 v = src[c];
+      for (int j = 0; j < top_k; ++j) {
+        const int r = __shfl_sync(0xffffffffu, my_row, j);
+        if (r >= 0) reinterpret_cast<uint4*>(xp + (size_t)r * H)[c] = v;
+      }
+    }
   }
 }
 
@@ -203,12 +206,12 @@ cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const v
                                                   o.row_of, o.tok_of, o.w_of, o.pos_of,
                                                   o.slot_stride, o.status);
   if (o.xp && x) {
-    const int R = T * top_k;
-    int grid = (R + 7) / 8;
-    const int cap = num_sms() * 16;
+    int grid = (T + 7) / 8;
+    const int cap = num_sms() * 8;
     if (grid > cap) grid = cap;
-    gather_rows_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), o.tok_of,
-                                                 R, H, T, static_cast<__nv_bfloat16*>(o.xp));
+    gather_tokens_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x),
+                                                   o.row_of, T, H, top_k,
+                                                   static_cast<__nv_bfloat16*>(o.xp));
   }
   return cudaGetLastError();
 }
