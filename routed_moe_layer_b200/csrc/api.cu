@@ -56,6 +56,11 @@ struct FwdLayout {
 // routed experts, then the shared expert.
 int slots_per_token(const moe_cfg_t& c) { return c.top_k + (c.I_shared > 0 ? 1 : 0); }
 
+// With I_shared == I the shared expert runs as one more group (number E) of
+// the routed grouped GEMMs: its rows follow the R routed rows in h, its A rows
+// come from x and its weights from ws13 / ws2.
+bool fuse_shared(const moe_cfg_t& c) { return c.I_shared > 0 && c.I_shared == c.I; }
+
 FwdLayout fwd_layout(const moe_cfg_t& c) {
   FwdLayout L;
   const size_t T = c.T, R = T * c.top_k, E = c.E;
@@ -66,8 +71,8 @@ FwdLayout fwd_layout(const moe_cfg_t& c) {
   L.ids = off;      off += align_up(R * 4);
   L.w = off;        off += align_up(R * 4);
   L.blk_hist = off; off += align_up(nblk * E * 4);
-  L.offsets = off;  off += align_up((E + 1) * 4);
-  L.mtiles = off;   off += align_up((E + 1) * 4);
+  L.offsets = off;  off += align_up((E + 2) * 4);
+  L.mtiles = off;   off += align_up((E + 2) * 4);
   L.row_of = off;   off += align_up(R * 4);
   L.tok_of = off;   off += align_up(R * 4);
   L.w_of = off;     off += align_up(R * 4);
@@ -75,8 +80,8 @@ FwdLayout fwd_layout(const moe_cfg_t& c) {
   // gathered expert rows [R, H]; once the up projection has read them, the same
   // bytes hold the weighted expert outputs in token-major slot order [T*slots, H]
   L.y = off;        off += align_up(std::max(R, T * (size_t)slots_per_token(c)) * c.H * 2);
-  L.h = off;        off += align_up(R * c.I * 2);
-  L.hs = off;       off += align_up(T * c.I_shared * 2);
+  L.h = off;        off += align_up((R + (fuse_shared(c) ? T : 0)) * c.I * 2);
+  L.hs = off;       off += align_up(fuse_shared(c) ? 0 : T * c.I_shared * 2);
   L.total = off;
   return L;
 }
@@ -239,17 +244,24 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
 
   // tensor maps (host-side descriptors, passed by value to the kernels)
   const int slots = slots_per_token(c);
-  CUtensorMap tm_xp, tm_w13, tm_h, tm_w2, tm_x, tm_ws13, tm_hs, tm_ws2;
+  const bool fused = fuse_shared(c);
+  const size_t h_rows = R + (fused ? T : 0);
+  CUtensorMap tm_xp, tm_w13, tm_h, tm_h_shared, tm_w2, tm_x, tm_ws13, tm_hs, tm_ws2;
   RMOE_TRY(make_tmap_2d(&tm_xp, xp, R, c.H));
-  RMOE_TRY(make_tmap_2d(&tm_x, x, T, c.H));
   RMOE_TRY(make_tmap_3d(&tm_w13, w13, c.E, 2 * (uint64_t)c.I, c.H));
   RMOE_TRY(make_tmap_2d(&tm_h, h, R, c.I));
+  // the shared group's rows of h (rows R..R+T-1), re-based to row 0
+  if (fused) RMOE_TRY(make_tmap_2d(&tm_h_shared, h + R * c.I, T, c.I));
   RMOE_TRY(make_tmap_3d(&tm_w2, w2, c.E, c.H, c.I));
   if (c.I_shared > 0) {
+    RMOE_TRY(make_tmap_2d(&tm_x, x, T, c.H));
     RMOE_TRY(make_tmap_3d(&tm_ws13, ws13, 1, 2 * (uint64_t)c.I_shared, c.H));
-    RMOE_TRY(make_tmap_2d(&tm_hs, hs, T, c.I_shared));
     RMOE_TRY(make_tmap_3d(&tm_ws2, ws2, 1, c.H, c.I_shared));
+    if (!fused) RMOE_TRY(make_tmap_2d(&tm_hs, hs, T, c.I_shared));
+  } else {
+    tm_x = tm_ws13 = tm_ws2 = tm_xp;  // unused second maps
   }
+  if (!fused) tm_h_shared = tm_h;  // unused
   const int sms = num_sms();
 
   auto record = [&](int i) -> cudaError_t {
@@ -272,23 +284,30 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
   o.w_of = at<float>(workspace, L.w_of);
   o.pos_of = at<int>(workspace, L.pos_of);
   o.slot_stride = slots;
+  o.extra_rows = fused ? c.T : 0;
   o.xp = xp;
   RMOE_TRY(launch_permute(ids, tw, x, c.T, c.H, c.E, c.top_k, o, s));
 
-  // tiles of MTILE rows, each computed by a pair of CTAs; every expert adds at
+  // tiles of MTILE rows, each computed by a pair of CTAs; every group adds at
   // most one partial tile
-  const int mt_bound = (int)(R / MTILE) + c.E;
+  const int groups = c.E + (fused ? 1 : 0);
+  const long long mt_bound = (long long)(h_rows / MTILE) + groups;
   GemmArgs a;
   memset(&a, 0, sizeof(a));
   a.status = status;
   a.timeout_ns = timeout;
+  a.alt_group = -1;
 
   RMOE_TRY(record(MOE_STAGE_EXPERT_UP));
-  {  // h = silu(xp . W13g^T) * (xp . W13u^T), per expert
+  {  // h = silu(A . W13g^T) * (A . W13u^T) per group: A = gathered rows (experts), x (shared)
     GemmArgs g = a;
     g.mtile_start = mtiles;
     g.row_start = offsets;
-    g.num_groups = c.E;
+    g.num_groups = groups;
+    if (fused) {
+      g.alt_group = c.E;
+      g.alt_row0 = (int)R;
+    }
     g.n_tiles = (c.I + 127) / 128;
     g.k_steps = c.H / 64;
     g.n_out_tile = 128;
@@ -297,14 +316,18 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
     g.ldo = c.I;
     g.n_valid = c.I;
     const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
-    RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_xp, tm_w13, g, grid, s));
+    RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_xp, tm_w13, tm_x, tm_ws13, g, grid, s));
   }
   RMOE_TRY(record(MOE_STAGE_EXPERT_DOWN));
-  {  // Y[t*slots + j] = w_tj * (h . W2^T), per expert
+  {  // Y[t*slots + j] = w_tj * (h . W2^T) per expert; shared rows to slot top_k, unscaled
     GemmArgs g = a;
     g.mtile_start = mtiles;
     g.row_start = offsets;
-    g.num_groups = c.E;
+    g.num_groups = groups;
+    if (fused) {
+      g.alt_group = c.E;
+      g.alt_row0 = (int)R;
+    }
     g.n_tiles = (c.H + 255) / 256;
     g.k_steps = c.I / 64;
     g.n_out_tile = 256;
@@ -314,11 +337,13 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
     g.n_valid = c.H;
     g.row_scale = o.w_of;
     g.dest_pos = o.pos_of;
+    g.dest_mul = slots;
+    g.dest_add = c.top_k;
     const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
-    RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, g, grid, s));
+    RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, tm_h_shared, tm_ws2, g, grid, s));
   }
   RMOE_TRY(record(MOE_STAGE_SHARED_EXPERT));
-  if (c.I_shared > 0) {
+  if (c.I_shared > 0 && !fused) {
     {  // hs = silu(x . Ws13g^T) * (x . Ws13u^T)
       GemmArgs g = a;
       g.single_rows = c.T;
@@ -330,7 +355,8 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
       g.ldo = c.I_shared;
       g.n_valid = c.I_shared;
       const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
-      RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_x, tm_ws13, g, std::min(sms, 2 * tiles), s));
+      RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_x, tm_ws13, tm_x, tm_ws13, g,
+                                   std::min(sms, 2 * tiles), s));
     }
     {  // Y[t*slots + top_k] = hs . Ws2^T  (unscaled)
       GemmArgs g = a;
@@ -345,7 +371,8 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
       g.dest_mul = slots;
       g.dest_add = c.top_k;
       const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
-      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_hs, tm_ws2, g, std::min(sms, 2 * tiles), s));
+      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_hs, tm_ws2, tm_hs, tm_ws2, g,
+                                   std::min(sms, 2 * tiles), s));
     }
   }
   RMOE_TRY(record(MOE_STAGE_COMBINE));

@@ -53,7 +53,7 @@ constexpr int B_BYTES = (BN / 2) * BK * 2;  // this CTA's half of the B tile
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 320;  // producer warp, MMA warp, 8 epilogue warps
 constexpr int EPI_THREADS = 256;
-constexpr int MAX_GROUPS = 128;
+constexpr int MAX_GROUPS = 129;  // 128 experts + the shared expert
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN);
 constexpr int EPI_WARPS = EPI_THREADS / 32;
@@ -136,8 +136,13 @@ __device__ __forceinline__ RowIn epilogue_row_inputs(const GemmArgs& a, const Ti
   if constexpr (EPI == EPI_ROWSCALE) {
     if (r_in_tile < tc.rows) {
       const int row = tc.row0 + r_in_tile;
-      in.w = a.row_scale ? a.row_scale[row] : 1.0f;
-      in.drow = a.dest_pos ? a.dest_pos[row] : row * a.dest_mul + a.dest_add;
+      if (tc.g == a.alt_group || !a.dest_pos) {  // unweighted rows at t*dest_mul + dest_add
+        in.w = 1.0f;
+        in.drow = (row - (tc.g == a.alt_group ? a.alt_row0 : 0)) * a.dest_mul + a.dest_add;
+      } else {
+        in.w = a.row_scale ? a.row_scale[row] : 1.0f;
+        in.drow = a.dest_pos[row];
+      }
     }
   }
   return in;
@@ -200,7 +205,9 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tbase,
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmA2,
+                        const __grid_constant__ CUtensorMap tmB2, const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -232,6 +239,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 32) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (args.alt_group >= 0) {
+      tma_prefetch_desc(&tmA2);
+      tma_prefetch_desc(&tmB2);
+    }
   }
   __syncthreads();
   const int total_m = args.mtile_start ? st.mt_start[args.num_groups]
@@ -259,8 +270,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       bool ok = true;
       for (int tile = cluster; ok && tile < total; tile += nclusters) {
         const TileCoord tc = tile_coord(tile, args, st.mt_start, st.row_start);
-        const int a_row = tc.row0 + BM * (int)rank;
+        const bool alt = tc.g == args.alt_group;
+        const CUtensorMap* ma = alt ? &tmA2 : &tmA;
+        const CUtensorMap* mb = alt ? &tmB2 : &tmB;
+        const int a_row = tc.row0 + BM * (int)rank - (alt ? args.alt_row0 : 0);
+        const int b_grp = alt ? 0 : tc.g;
         const int b_row = tc.nt * args.n_out_tile + (int)rank * args.b_second;
+        // a CTA whose half of the tile holds no rows of the group skips its A
+        // load (its accumulator rows are never stored); the leader arms the
+        // barrier for the bytes that will actually arrive
+        const bool load_a = tc.rows > BM * (int)rank;
+        const uint32_t tx = 2 * B_BYTES + A_BYTES + (tc.rows > BM ? A_BYTES : 0);
         for (int ks = 0; ks < args.k_steps; ++ks) {
           if (!mbar_wait(&st.empty[stage], phase ^ 1u, wc, 10)) {
             ok = false;
@@ -268,9 +288,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
           uint8_t* sa = smem + (size_t)stage * STAGE_BYTES;
           const uint32_t full_leader = mapa_shared(smem_u32(&st.full[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(&st.full[stage], 2 * STAGE_BYTES);
-          tma_load_2d_pair(sa, &tmA, full_leader, ks * BK, a_row);
-          tma_load_3d_pair(sa + A_BYTES, &tmB, full_leader, ks * BK, b_row, tc.g);
+          if (leader) mbar_arrive_expect_tx(&st.full[stage], tx);
+          if (load_a) tma_load_2d_pair(sa, ma, full_leader, ks * BK, a_row);
+          tma_load_3d_pair(sa + A_BYTES, mb, full_leader, ks * BK, b_row, b_grp);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -375,14 +395,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 template <int EPI>
-cudaError_t launch_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args,
-                       int grid, cudaStream_t stream) {
+cudaError_t launch_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
+                       const CUtensorMap& tmB2, const GemmArgs& args, int grid,
+                       cudaStream_t stream) {
   static cudaError_t attr = cudaFuncSetAttribute(
       grouped_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (attr != cudaSuccess) return attr;
   grid &= ~1;  // clusters of two CTAs
   if (grid < 2) grid = 2;
-  grouped_gemm_kernel<EPI><<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, args);
+  grouped_gemm_kernel<EPI><<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmA2, tmB2, args);
   return cudaGetLastError();
 }
 
@@ -418,13 +439,14 @@ cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, uint64_t groups, ui
 }
 
 cudaError_t launch_grouped_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                const CUtensorMap& tmA2, const CUtensorMap& tmB2,
                                 const GemmArgs& args, int grid, cudaStream_t stream) {
   if (args.mtile_start && args.num_groups > MAX_GROUPS) return cudaErrorInvalidValue;
   switch (epi) {
     case EPI_SWIGLU:
-      return launch_epi<EPI_SWIGLU>(tmA, tmB, args, grid, stream);
+      return launch_epi<EPI_SWIGLU>(tmA, tmB, tmA2, tmB2, args, grid, stream);
     case EPI_ROWSCALE:
-      return launch_epi<EPI_ROWSCALE>(tmA, tmB, args, grid, stream);
+      return launch_epi<EPI_ROWSCALE>(tmA, tmB, tmA2, tmB2, args, grid, stream);
     default:
       return cudaErrorInvalidValue;
   }

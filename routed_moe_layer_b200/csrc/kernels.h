@@ -33,6 +33,8 @@ struct PermuteOut {
   int* tok_of;          // [T*k]
   int* pos_of = nullptr;  // [T*k] or null: slot position t*slot_stride + j of each row
   int slot_stride = 0;    // slots per token in the token-major output buffer
+  int extra_rows = 0;     // > 0: one more group of this many rows after the experts
+                          // (expert_offsets / mtile_start then have E+2 entries)
   float* w_of;          // [T*k] or null
   void* xp;             // [T*k, H] bf16 or null
 };
@@ -49,6 +51,8 @@ struct GemmArgs {
   const int* row_start;    // [num_groups+1] device first row of each group
   int num_groups;
   int single_rows;         // rows of the only group when mtile_start == null
+  int alt_group;           // group read through the second pair of maps (-1: none); its
+  int alt_row0;            //   rows start at alt_row0 in the first A map's row numbering
   int n_tiles;             // output tiles along N
   int k_steps;             // K / 64
   int n_out_tile;          // output columns per tile: 128 (SwiGLU) or 256
@@ -70,7 +74,9 @@ cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint
 cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, uint64_t groups, uint64_t n_rows,
                          uint64_t K);
 
+// tmA2/tmB2 serve group args.alt_group (A rows re-based to 0, B group 0).
 cudaError_t launch_grouped_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                const CUtensorMap& tmA2, const CUtensorMap& tmB2,
                                 const GemmArgs& args, int grid, cudaStream_t stream);
 
 int num_sms();

@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(PT)
 
 // One CTA of 1024 threads: expert e = tid % E, chunk ch = tid / E of the blocks.
 __global__ void __launch_bounds__(1024)
-    permute_scan_kernel(int* __restrict__ blk_hist, int nblk, int E,
+    permute_scan_kernel(int* __restrict__ blk_hist, int nblk, int E, int extra_rows,
                         int* __restrict__ expert_offsets, int* __restrict__ mtile_start) {
   __shared__ int part[1024];
   __shared__ int excl_rows[MAXE + 1];
@@ -125,6 +125,10 @@ __global__ void __launch_bounds__(1024)
   if (tid <= E) {
     expert_offsets[tid] = excl_rows[tid];
     if (mtile_start) mtile_start[tid] = excl_tiles[tid];
+  }
+  if (tid == 0 && extra_rows > 0) {  // one more group after the experts
+    expert_offsets[E + 1] = excl_rows[E] + extra_rows;
+    if (mtile_start) mtile_start[E + 1] = excl_tiles[E] + (extra_rows + MTILE - 1) / MTILE;
   }
   if (active) {
     int run = excl_rows[e] + part[ch * E + e];
@@ -200,8 +204,8 @@ cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const v
                            int H, int E, int top_k, const PermuteOut& o, cudaStream_t stream) {
   const int nblk = (T + PT - 1) / PT;
   permute_count_kernel<<<nblk, PT, 0, stream>>>(topk_ids, T, E, top_k, o.blk_hist, o.status);
-  permute_scan_kernel<<<1, 1024, 0, stream>>>(o.blk_hist, nblk, E, o.expert_offsets,
-                                              o.mtile_start);
+  permute_scan_kernel<<<1, 1024, 0, stream>>>(o.blk_hist, nblk, E, o.extra_rows,
+                                              o.expert_offsets, o.mtile_start);
   permute_scatter_kernel<<<nblk, PT, 0, stream>>>(topk_ids, topk_w, T, E, top_k, o.blk_hist,
                                                   o.row_of, o.tok_of, o.w_of, o.pos_of,
                                                   o.slot_stride, o.status);
