@@ -173,10 +173,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tbase,
           const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
           pk[i] = pack_bf16x2(h0, h1);
         }
-        uint4* dst = reinterpret_cast<uint4*>(a.out + (size_t)row * a.ldo + col0 + c);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        // 64 bytes of the row as two full-sector stores
+        __nv_bfloat16* dst = a.out + (size_t)row * a.ldo + col0 + c;
+        st_global_v8(dst, pk);
+        st_global_v8(dst + 16, pk + 8);
       }
     }
   } else {  // EPI_ROWSCALE: weighted rows scattered to their token-major slot
@@ -193,10 +193,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tbase,
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           pk[i] = pack_bf16x2(w * __uint_as_float(v[2 * i]), w * __uint_as_float(v[2 * i + 1]));
-        uint4* dst = reinterpret_cast<uint4*>(a.out + (size_t)drow * a.ldo + col0 + c);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        // 64 bytes of the row as two full-sector stores
+        __nv_bfloat16* dst = a.out + (size_t)drow * a.ldo + col0 + c;
+        st_global_v8(dst, pk);
+        st_global_v8(dst + 16, pk + 8);
       }
     }
   }
