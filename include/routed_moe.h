@@ -71,7 +71,7 @@ typedef struct {
   int32_t I;                      /* moe_intermediate_size; multiple of 64 */
   int32_t I_shared;               /* shared expert intermediate size; 0 = none, else multiple of 64 */
   int32_t top_k;                  /* experts per token; 1..16 */
-  int32_t n_group;                /* expert groups */
+  int32_t n_group;                /* expert groups; 1..16 */
   int32_t topk_group;             /* groups kept per token */
   float routed_scaling_factor;    /* applied once, inside the router */
   int32_t norm_topk_prob;         /* 1: renormalise the chosen scores to sum 1 first */

@@ -20,7 +20,7 @@ constexpr size_t WS_ALIGN = 256;
 constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s
 constexpr int MAX_E = 128;
 constexpr int MAX_TOPK = 16;
-constexpr int MAX_NGROUP = 32;
+constexpr int MAX_NGROUP = 16;  // the router ranks groups within a half warp
 constexpr int MAX_DIM = 16384;
 
 size_t align_up(size_t v) { return (v + WS_ALIGN - 1) & ~(WS_ALIGN - 1); }

@@ -11,14 +11,15 @@
 // logits = x.hi^T + x.mid^T + x.lo^T accumulate in fp32 in TMEM -- an fp32 dot
 // product of the bf16 token and the fp32 router row, up to summation order.
 //   1. router_split_kernel    Wr [E,H] fp32 -> Wr3 [3,E,H] bf16
-//   2. router_gemm_kernel     tcgen05 128 tokens x 128 experts tiles, K split
-//                             into a number of chunks that depends on H only
-//                             (so a token's logits never depend on T); each
-//                             chunk's fp32 partial goes to [S,T,E]
-//   3. router_select_kernel   one warp per token: sums the S partials in order,
-//                             then sigmoid, bias, group top-2 sums, group
-//                             selection, expert selection and weights with
-//                             warp shuffles.
+//   2. router_gemm_kernel     persistent tcgen05 GEMM over items of 128 tokens x
+//                             128 experts x one K chunk; the number of chunks
+//                             depends on H only (so a token's logits never
+//                             depend on T); each chunk's fp32 partial goes to
+//                             [S,T,E]
+//   3. router_select_kernel   16 lanes per token (two tokens per warp): sums the
+//                             S partials in order, then sigmoid, bias, group
+//                             top-2 sums, group selection, expert selection
+//                             and weights with shuffles.
 #include <float.h>
 #include <limits.h>
 
@@ -38,13 +39,14 @@ constexpr int R_A_BYTES = RBM * RBK * 2;
 constexpr int R_B_BYTES = RBN * RBK * 2;
 constexpr int R_STAGE_BYTES = R_A_BYTES + 3 * R_B_BYTES;
 constexpr int R_THREADS = 192;
-constexpr uint32_t R_TMEM_COLS = 128;
+constexpr uint32_t R_TMEM_COLS = 256;  // two 128-column accumulators
 constexpr uint32_t R_IDESC = idesc_bf16_f32(RBM, RBN);
 
 struct __align__(8) RouterTail {
   uint64_t full[RSTAGES];
   uint64_t empty[RSTAGES];
-  uint64_t tfull;
+  uint64_t tfull[2];
+  uint64_t tempty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -75,7 +77,10 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// grid (m_tiles, S): tile blockIdx.x of 128 tokens, K chunk blockIdx.y.
+// Persistent: CTA b handles items b, b + gridDim.x, ... of the m_tiles x S
+// items (item = token tile * S + K chunk); two TMEM accumulators let the
+// epilogue of one item overlap the MMAs of the next, and the load pipeline
+// runs across items.
 __global__ void __launch_bounds__(R_THREADS, 1)
     router_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmW3, int T, int E, int k_steps,
@@ -86,17 +91,17 @@ __global__ void __launch_bounds__(R_THREADS, 1)
                                              ~static_cast<uintptr_t>(1023));
   RouterTail& st = *reinterpret_cast<RouterTail*>(smem + (size_t)RSTAGES * R_STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * RBM;
-  const int s = blockIdx.y;
-  const int kb = (int)((long long)s * k_steps / S), ke = (int)((long long)(s + 1) * k_steps / S);
-  const int nk = ke - kb;
+  const int items = ((T + RBM - 1) / RBM) * S;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < RSTAGES; ++i) {
       mbar_init(&st.full[i], 1);
       mbar_init(&st.empty[i], 1);
     }
-    mbar_init(&st.tfull, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&st.tfull[b], 1);
+      mbar_init(&st.tempty[b], 128);
+    }
     mbar_init(&st.drain, 1);
     st.abort_flag = 0;
     fence_mbar_init();
@@ -117,24 +122,33 @@ __global__ void __launch_bounds__(R_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;
       bool ok = true;
-      for (int i = 0; i < nk; ++i) {
-        const int stage = i % RSTAGES;
-        const uint32_t phase = (i / RSTAGES) & 1u;
-        if (!mbar_wait(&st.empty[stage], phase ^ 1u, wc, 40)) {
-          ok = false;
-          break;
-        }
-        uint8_t* sa = smem + (size_t)stage * R_STAGE_BYTES;
-        mbar_arrive_expect_tx(&st.full[stage], R_STAGE_BYTES);
-        const int kc = (kb + i) * RBK;
-        tma_load_2d(sa, &tmX, &st.full[stage], kc, m0);
+      for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
+        const int m0 = (it / S) * RBM, s = it % S;
+        const int kb = (int)((long long)s * k_steps / S);
+        const int ke = (int)((long long)(s + 1) * k_steps / S);
+        for (int k = kb; k < ke; ++k) {
+          if (!mbar_wait(&st.empty[stage], phase ^ 1u, wc, 40)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + (size_t)stage * R_STAGE_BYTES;
+          mbar_arrive_expect_tx(&st.full[stage], R_STAGE_BYTES);
+          tma_load_2d(sa, &tmX, &st.full[stage], k * RBK, m0);
 #pragma unroll
-        for (int t = 0; t < 3; ++t)
-          tma_load_3d(sa + R_A_BYTES + t * R_B_BYTES, &tmW3, &st.full[stage], kc, 0, t);
-        armed |= 1u << stage;
-        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          for (int t = 0; t < 3; ++t)
+            tma_load_3d(sa + R_A_BYTES + t * R_B_BYTES, &tmW3, &st.full[stage], k * RBK, 0, t);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == RSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
       }
       if (!ok) {
         for (int i = 0; i < RSTAGES; ++i)
@@ -143,50 +157,72 @@ __global__ void __launch_bounds__(R_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
       bool ok = true;
-      for (int i = 0; i < nk; ++i) {
-        const int stage = i % RSTAGES;
-        const uint32_t phase = (i / RSTAGES) & 1u;
-        if (!mbar_wait(&st.full[stage], phase, wc, 41)) {
-          ok = false;
-          break;
-        }
+      for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
+        const int s = it % S;
+        const int kb = (int)((long long)s * k_steps / S);
+        const int ke = (int)((long long)(s + 1) * k_steps / S);
+        if (!mbar_wait(&st.tempty[acc], acc_phase ^ 1u, wc, 43)) break;
         tc_fence_after_sync();
-        const uint32_t sa = smem_u32(smem + (size_t)stage * R_STAGE_BYTES);
-        const uint64_t da = sdesc_kmajor_sw128(sa);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * RBN);
+        for (int k = kb; k < ke; ++k) {
+          if (!mbar_wait(&st.full[stage], phase, wc, 41)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t sa = smem_u32(smem + (size_t)stage * R_STAGE_BYTES);
+          const uint64_t da = sdesc_kmajor_sw128(sa);
 #pragma unroll
-        for (int t = 0; t < 3; ++t) {
-          const uint64_t db = sdesc_kmajor_sw128(sa + R_A_BYTES + t * R_B_BYTES);
+          for (int t = 0; t < 3; ++t) {
+            const uint64_t db = sdesc_kmajor_sw128(sa + R_A_BYTES + t * R_B_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < RBK / 16; ++kk)
-            umma_bf16_ss(tmem_base, da + 2 * kk, db + 2 * kk, R_IDESC,
-                         (i | t | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < RBK / 16; ++kk)
+              umma_bf16_ss(d_tmem, da + 2 * kk, db + 2 * kk, R_IDESC,
+                           (k != kb || t != 0 || kk != 0) ? 1u : 0u);
+          }
+          umma_commit(&st.empty[stage]);
+          if (++stage == RSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
-        umma_commit(&st.empty[stage]);
+        if (!ok) break;
+        umma_commit(&st.tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
       }
-      if (ok) umma_commit(&st.tfull);
       umma_commit(&st.drain);
       wait_drain(&st.drain, 0, timeout_ns);
     }
   } else {
+    // ------------------------------------------------ epilogue warps 2..5
     const int q = warp & 3;
-    const bool ok = mbar_wait(&st.tfull, 0, wc, 42);
-    if (__all_sync(FULL, ok)) {
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int it = blockIdx.x; it < items; it += gridDim.x) {
+      const int m0 = (it / S) * RBM, s = it % S;
+      const bool ok = mbar_wait(&st.tfull[acc], acc_phase, wc, 42);
+      if (!__all_sync(FULL, ok)) break;
       tc_fence_after_sync();
       const int row = m0 + q * 32 + lane;
       float* dst = partial + ((size_t)s * T + row) * E;
+      const uint32_t tbase =
+          tmem_base + static_cast<uint32_t>(acc * RBN) + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
       for (int c = 0; c < RBN; c += 32) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + c, v);
+        tmem_ld_32x32b_x32(tbase + c, v);
         tmem_ld_wait();
         if (row < T && c < E) {
-          if (c + 32 <= E && (E & 3) == 0) {
+          if (c + 32 <= E && (E & 7) == 0) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              reinterpret_cast<float4*>(dst + c)[i] =
-                  make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                              __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            for (int i = 0; i < 4; ++i) st_global_v8(dst + c + 8 * i, v + 8 * i);
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
@@ -194,6 +230,10 @@ __global__ void __launch_bounds__(R_THREADS, 1)
           }
         }
       }
+      tc_fence_before_sync();
+      mbar_arrive(&st.tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
     }
   }
 
@@ -205,10 +245,11 @@ __global__ void __launch_bounds__(R_THREADS, 1)
   }
 }
 
-// Warp-wide argmax: larger value wins, equal values go to the lower index.
-__device__ __forceinline__ void warp_argmax(float& v, int& idx) {
+// Argmax over the 16 lanes of a half warp: larger value wins, equal values
+// go to the lower index.
+__device__ __forceinline__ void half_argmax(float& v, int& idx) {
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
+  for (int off = 8; off > 0; off >>= 1) {
     const float ov = __shfl_xor_sync(FULL, v, off);
     const int oi = __shfl_xor_sync(FULL, idx, off);
     if (ov > v || (ov == v && oi < idx)) {
@@ -218,35 +259,41 @@ __device__ __forceinline__ void warp_argmax(float& v, int& idx) {
   }
 }
 
-// One warp per token; lane l holds experts l + 32*i.
+// Two tokens per warp: lanes 0-15 take one token, lanes 16-31 the next; sub-
+// lane l of a half holds experts l + 16*i (i < 8).
 constexpr int SEL_WARPS = 8;
+constexpr int SEL_LPT = 16;                // lanes per token
+constexpr int SEL_NE = RBN / SEL_LPT;      // experts per lane
 
 __global__ void __launch_bounds__(SEL_WARPS * 32)
     router_select_kernel(const float* __restrict__ partial, int S, const float* __restrict__ bias,
                          RouterParams p, int32_t* __restrict__ topk_ids,
                          float* __restrict__ topk_w) {
-  constexpr int NE = RBN / 32;
-  __shared__ float sc[SEL_WARPS][RBN];  // bias-corrected scores of the warp's token
+  __shared__ float sc[SEL_WARPS * 2][RBN];  // bias-corrected scores of each token
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int warps = gridDim.x * SEL_WARPS;
+  const int half = lane >> 4, sl = lane & 15;
   const int T = p.T, E = p.E;
   const int gs = E / p.n_group;
   const bool group_step = p.topk_group < p.n_group;
-  float b[NE];
-  int grp[NE];  // group of each held expert (computed once)
+  float* my_sc = sc[wib * 2 + half];
+  float b[SEL_NE];
+  int grp[SEL_NE];
 #pragma unroll
-  for (int i = 0; i < NE; ++i) {
-    const int e = lane + 32 * i;
+  for (int i = 0; i < SEL_NE; ++i) {
+    const int e = sl + SEL_LPT * i;
     b[i] = (e < E) ? bias[e] : 0.f;
     grp[i] = (e < E) ? e / gs : 0;
   }
-  for (int t = blockIdx.x * SEL_WARPS + wib; t < T; t += warps) {
-    float s[NE], c[NE];
-    bool avail[NE];
+  const int pairs = (T + 1) / 2;
+  for (int pr = blockIdx.x * SEL_WARPS + wib; pr < pairs; pr += gridDim.x * SEL_WARPS) {
+    const int t = 2 * pr + half;
+    const bool tok_ok = t < T;
+    float s[SEL_NE], c[SEL_NE];
+    bool avail[SEL_NE];
 #pragma unroll
-    for (int i = 0; i < NE; ++i) {
-      const int e = lane + 32 * i;
-      avail[i] = e < E;
+    for (int i = 0; i < SEL_NE; ++i) {
+      const int e = sl + SEL_LPT * i;
+      avail[i] = tok_ok && e < E;
       float l = 0.f;
       if (avail[i]) {
         l = partial[(size_t)t * E + e];
@@ -257,14 +304,14 @@ __global__ void __launch_bounds__(SEL_WARPS * 32)
     }
     if (group_step) {
 #pragma unroll
-      for (int i = 0; i < NE; ++i)
-        if (avail[i]) sc[wib][lane + 32 * i] = c[i];
+      for (int i = 0; i < SEL_NE; ++i)
+        if (avail[i]) my_sc[sl + SEL_LPT * i] = c[i];
       __syncwarp();
-      // lane j < n_group: group score = sum of the two largest c of group j
+      // sub-lane j < n_group: group score = sum of the two largest c of group j
       float G = -FLT_MAX;
-      if (lane < p.n_group) {
+      if (tok_ok && sl < p.n_group) {
         float v1 = -FLT_MAX, v2 = -FLT_MAX;
-        const float* g = &sc[wib][lane * gs];
+        const float* g = my_sc + sl * gs;
         for (int q = 0; q < gs; ++q) {
           const float v = g[q];
           if (v > v1) {
@@ -276,15 +323,16 @@ __global__ void __launch_bounds__(SEL_WARPS * 32)
         }
         G = v1 + v2;
       }
-      // rank of each group: larger score first, ties to the lower group index
+      // rank of each group in its half: larger score first, ties to the lower group
       int rank = 0;
       for (int m = 0; m < p.n_group; ++m) {
-        const float Gm = __shfl_sync(FULL, G, m);
-        if (Gm > G || (Gm == G && m < lane)) ++rank;
+        const float Gm = __shfl_sync(FULL, G, (lane & 16) | m);
+        if (Gm > G || (Gm == G && m < sl)) ++rank;
       }
-      const uint32_t kept = __ballot_sync(FULL, lane < p.n_group && rank < p.topk_group);
+      const uint32_t kept =
+          (__ballot_sync(FULL, sl < p.n_group && rank < p.topk_group) >> (16 * half)) & 0xFFFFu;
 #pragma unroll
-      for (int i = 0; i < NE; ++i)
+      for (int i = 0; i < SEL_NE; ++i)
         if (avail[i] && !((kept >> grp[i]) & 1u)) avail[i] = false;
       __syncwarp();
     }
@@ -295,24 +343,24 @@ __global__ void __launch_bounds__(SEL_WARPS * 32)
       float v = -FLT_MAX;
       int idx = INT_MAX;
 #pragma unroll
-      for (int i = 0; i < NE; ++i) {
-        const int e = lane + 32 * i;
+      for (int i = 0; i < SEL_NE; ++i) {
+        const int e = sl + SEL_LPT * i;
         if (avail[i] && (c[i] > v || (c[i] == v && e < idx))) {
           v = c[i];
           idx = e;
         }
       }
-      warp_argmax(v, idx);
-      const int owner = idx & 31, slot = (idx >> 5) & (NE - 1);
+      half_argmax(v, idx);
+      const int owner = idx & (SEL_LPT - 1), slot = (idx >> 4) & (SEL_NE - 1);
       float sv = s[0];
 #pragma unroll
-      for (int i = 1; i < NE; ++i)
+      for (int i = 1; i < SEL_NE; ++i)
         if (slot == i) sv = s[i];
-      sv = __shfl_sync(FULL, sv, owner);
+      sv = __shfl_sync(FULL, sv, (lane & 16) | owner);
       if (idx < E) {
-        if (lane == owner) {
+        if (sl == owner) {
 #pragma unroll
-          for (int i = 0; i < NE; ++i)
+          for (int i = 0; i < SEL_NE; ++i)
             if (slot == i) avail[i] = false;
         }
       } else {
@@ -320,15 +368,15 @@ __global__ void __launch_bounds__(SEL_WARPS * 32)
         idx = -1;  // no candidate left (non-finite scores); the permutation reports it
       }
       sum += sv;
-      if (lane == r) {
+      if (sl == r) {
         my_id = idx;
         my_s = sv;
       }
     }
-    if (lane < p.top_k) {
+    if (tok_ok && sl < p.top_k) {
       const float wv = p.norm_topk_prob ? p.rsf * (my_s / sum) : p.rsf * my_s;
-      topk_ids[(size_t)t * p.top_k + lane] = my_id;
-      topk_w[(size_t)t * p.top_k + lane] = wv;
+      topk_ids[(size_t)t * p.top_k + sl] = my_id;
+      topk_w[(size_t)t * p.top_k + sl] = wv;
     }
   }
 }
@@ -364,10 +412,11 @@ cudaError_t launch_router(const void* x, const float* Wr, const float* bias, con
                              (int)R_SMEM_BYTES);
   if (err != cudaSuccess) return err;
   const int S = router_splits(H);
-  const dim3 grid((T + RBM - 1) / RBM, S);
+  const int items = ((T + RBM - 1) / RBM) * S;
+  const int grid = items < num_sms() ? items : num_sms();
   router_gemm_kernel<<<grid, R_THREADS, R_SMEM_BYTES, stream>>>(tmX, tmW3, T, E, H / RBK, S,
                                                                  partial, status, timeout_ns);
-  int sel_grid = (T + SEL_WARPS - 1) / SEL_WARPS;
+  int sel_grid = ((T + 1) / 2 + SEL_WARPS - 1) / SEL_WARPS;
   const int cap = num_sms() * 16;
   if (sel_grid > cap) sel_grid = cap;
   router_select_kernel<<<sel_grid, SEL_WARPS * 32, 0, stream>>>(partial, S, bias, p, topk_ids,

@@ -61,7 +61,8 @@ DEFAULT = BlockConfig(T=19412, H=2048)
     ({"topk_group": 5}, 1),                 # more kept groups than groups
     ({"n_group": 64, "topk_group": 2}, 1),  # 2 experts per group * 2 groups < top_k
     ({"n_group": 128, "topk_group": 64}, 1),  # groups of one expert cannot give a top-2
-    ({"n_group": 128, "topk_group": 128}, 2),  # no group step, but n_group > 32
+    ({"n_group": 128, "topk_group": 128}, 2),  # no group step, but n_group > 16
+    ({"n_group": 32, "topk_group": 8}, 2),     # more groups than a half warp ranks
     ({"top_k": 17, "topk_group": 4}, 2),
     ({"H": 1000}, 2),
     ({"I": 96}, 2),
