@@ -93,8 +93,10 @@ typedef struct {
                              may be the same buffer as out */
   int32_t* topk_ids;      /* device int32 [T,top_k] or NULL: also write the routing ids */
   float* topk_w;          /* device fp32 [T,top_k] or NULL: also write the routing weights */
-  void** stage_events;    /* host array of MOE_NUM_STAGES+1 cudaEvent_t or NULL: event i is
-                             recorded on stream before stage i, the last one after the last */
+  void** stage_events;    /* host array of MOE_NUM_STAGES+1 cudaEvent_t or NULL: event i (if
+                             not NULL) is recorded on stream before stage i, the last one after
+                             the last stage.  Each recorded event orders the kernels around it
+                             strictly, so record only the boundaries you time. */
   int64_t wait_timeout_ns;/* limit of every device-side wait; 0 = 2 s */
 } moe_forward_opts_t;
 

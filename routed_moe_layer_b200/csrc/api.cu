@@ -178,7 +178,6 @@ int32_t moe_route(const void* x, const float* Wr, const float* bias, const moe_c
   if (!ws_ok(workspace, workspace_bytes, moe_route_workspace_bytes(cfg))) return MOE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* status = at<int>(workspace, 0);
-  RMOE_TRY(launch_status_reset(status, s));
   return cuda_status(launch_router(x, Wr, bias, router_params(*cfg), topk_ids, topk_w,
                                    at<void>(workspace, align_up(sizeof(DevStatus))), status,
                                    DEFAULT_TIMEOUT_NS, s));
@@ -265,11 +264,10 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
   const int sms = num_sms();
 
   auto record = [&](int i) -> cudaError_t {
-    return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
+    return (ev && ev[i]) ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
   };
 
   RMOE_TRY(record(MOE_STAGE_ROUTER));
-  RMOE_TRY(launch_status_reset(status, s));
   RMOE_TRY(launch_router(x, Wr, bias, router_params(c), ids, tw, at<void>(workspace, L.router),
                          status, timeout, s));
 

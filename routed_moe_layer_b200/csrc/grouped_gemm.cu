@@ -208,6 +208,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmA2,
                         const __grid_constant__ CUtensorMap tmB2, const GemmArgs args) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -403,8 +405,8 @@ cudaError_t launch_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUt
   if (attr != cudaSuccess) return attr;
   grid &= ~1;  // clusters of two CTAs
   if (grid < 2) grid = 2;
-  grouped_gemm_kernel<EPI><<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmA2, tmB2, args);
-  return cudaGetLastError();
+  return launch_chained(grouped_gemm_kernel<EPI>, dim3(grid), dim3(THREADS), SMEM_BYTES, stream,
+                        tmA, tmB, tmA2, tmB2, args);
 }
 
 }  // namespace

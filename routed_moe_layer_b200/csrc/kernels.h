@@ -5,7 +5,28 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace rmoe {
+
+// Launches kernel k chained to the previous work of the stream (programmatic
+// stream serialisation; the kernel itself waits with pdl_wait before reading
+// what its predecessors wrote).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
 
 struct RouterParams {
   int T, H, E, top_k, n_group, topk_group, norm_topk_prob;
@@ -16,6 +37,7 @@ struct RouterParams {
 // fp32 partial logits of the K chunks (router_scratch_bytes).
 int router_splits(int H);
 size_t router_scratch_bytes(int T, int H, int E);
+// Also clears the status word (the first kernel of a forward).
 cudaError_t launch_router(const void* x, const float* Wr, const float* bias, const RouterParams& p,
                           int32_t* topk_ids, float* topk_w, void* scratch, int* status,
                           unsigned long long timeout_ns, cudaStream_t stream);

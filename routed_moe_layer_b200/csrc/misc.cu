@@ -12,6 +12,8 @@ namespace {
 __global__ void __launch_bounds__(256)
     rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ gamma, float eps,
                    int T, int H, __nv_bfloat16* __restrict__ xn) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= T) return;
@@ -58,6 +60,8 @@ __global__ void __launch_bounds__(256)
                          int top_k, int T, int H, int slots,
                          const __nv_bfloat16* __restrict__ residual,
                          __nv_bfloat16* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (blockDim.x >> 5);
   for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
@@ -121,9 +125,9 @@ __global__ void selftest_wait_kernel(int* status, unsigned long long timeout_ns)
 cudaError_t launch_rmsnorm(const void* x, const float* gamma, float eps, int T, int H, void* xn,
                            cudaStream_t stream) {
   const int grid = (T + 7) / 8;
-  rmsnorm_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), gamma, eps, T,
-                                           H, static_cast<__nv_bfloat16*>(xn));
-  return cudaGetLastError();
+  return launch_chained(rmsnorm_kernel, dim3(grid), dim3(256), 0, stream,
+                        static_cast<const __nv_bfloat16*>(x), gamma, eps, T, H,
+                        static_cast<__nv_bfloat16*>(xn));
 }
 
 cudaError_t launch_combine_slots(const void* Y, const int* row_of, int top_k, int T, int H,
@@ -131,10 +135,10 @@ cudaError_t launch_combine_slots(const void* Y, const int* row_of, int top_k, in
   int grid = (T + 7) / 8;
   const int cap = num_sms() * 8;
   if (grid > cap) grid = cap;
-  combine_slots_kernel<<<grid, 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(Y), row_of, top_k, T, H, slots,
-      static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError();
+  return launch_chained(combine_slots_kernel, dim3(grid), dim3(256), 0, stream,
+                        static_cast<const __nv_bfloat16*>(Y), row_of, top_k, T, H, slots,
+                        static_cast<const __nv_bfloat16*>(residual),
+                        static_cast<__nv_bfloat16*>(out));
 }
 
 cudaError_t launch_status_reset(int* status, cudaStream_t stream) {

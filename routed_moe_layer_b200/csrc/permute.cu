@@ -46,6 +46,8 @@ __global__ void __launch_bounds__(PT)
     permute_count_kernel(const int32_t* __restrict__ ids, int T, int E, int top_k,
                          int* __restrict__ blk_hist, int* status) {
   __shared__ uint32_t masks[PW][MAXE];
+  pdl_launch_dependents();
+  pdl_wait();
   build_masks(ids, T, E, top_k, masks, status);
   for (int e = threadIdx.x; e < E; e += PT) {
     int cnt = 0;
@@ -62,6 +64,8 @@ __global__ void __launch_bounds__(1024)
   __shared__ int part[1024];
   __shared__ int excl_rows[MAXE + 1];
   __shared__ int excl_tiles[MAXE + 1];
+  pdl_launch_dependents();
+  pdl_wait();
   const int tid = threadIdx.x;
   const int C = 1024 / E;
   const int e = tid % E, ch = tid / E;
@@ -149,6 +153,8 @@ __global__ void __launch_bounds__(PT)
                            int* status) {
   __shared__ uint32_t masks[PW][MAXE];
   __shared__ int wbase[PW][MAXE];
+  pdl_launch_dependents();
+  pdl_wait();
   build_masks(ids, T, E, top_k, masks, status);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int e = tid; e < E; e += PT) {
@@ -183,6 +189,8 @@ __global__ void __launch_bounds__(PT)
 __global__ void __launch_bounds__(256)
     gather_tokens_kernel(const __nv_bfloat16* __restrict__ x, const int* __restrict__ row_of,
                          int T, int H, int top_k, __nv_bfloat16* __restrict__ xp) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (blockDim.x >> 5);
   for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
@@ -203,19 +211,24 @@ __global__ void __launch_bounds__(256)
 cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const void* x, int T,
                            int H, int E, int top_k, const PermuteOut& o, cudaStream_t stream) {
   const int nblk = (T + PT - 1) / PT;
-  permute_count_kernel<<<nblk, PT, 0, stream>>>(topk_ids, T, E, top_k, o.blk_hist, o.status);
-  permute_scan_kernel<<<1, 1024, 0, stream>>>(o.blk_hist, nblk, E, o.extra_rows,
-                                              o.expert_offsets, o.mtile_start);
-  permute_scatter_kernel<<<nblk, PT, 0, stream>>>(topk_ids, topk_w, T, E, top_k, o.blk_hist,
-                                                  o.row_of, o.tok_of, o.w_of, o.pos_of,
-                                                  o.slot_stride, o.status);
+  cudaError_t err = launch_chained(permute_count_kernel, dim3(nblk), dim3(PT), 0, stream, topk_ids,
+                                   T, E, top_k, o.blk_hist, o.status);
+  if (err != cudaSuccess) return err;
+  err = launch_chained(permute_scan_kernel, dim3(1), dim3(1024), 0, stream, o.blk_hist, nblk, E,
+                       o.extra_rows, o.expert_offsets, o.mtile_start);
+  if (err != cudaSuccess) return err;
+  err = launch_chained(permute_scatter_kernel, dim3(nblk), dim3(PT), 0, stream, topk_ids, topk_w,
+                       T, E, top_k, (const int*)o.blk_hist, o.row_of, o.tok_of, o.w_of, o.pos_of,
+                       o.slot_stride, o.status);
+  if (err != cudaSuccess) return err;
   if (o.xp && x) {
     int grid = (T + 7) / 8;
     const int cap = num_sms() * 8;
     if (grid > cap) grid = cap;
-    gather_tokens_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x),
-                                                   o.row_of, T, H, top_k,
-                                                   static_cast<__nv_bfloat16*>(o.xp));
+    err = launch_chained(gather_tokens_kernel, dim3(grid), dim3(256), 0, stream,
+                         static_cast<const __nv_bfloat16*>(x), (const int*)o.row_of, T, H, top_k,
+                         static_cast<__nv_bfloat16*>(o.xp));
+    if (err != cudaSuccess) return err;
   }
   return cudaGetLastError();
 }

@@ -63,7 +63,14 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, uint6
 }
 
 __global__ void __launch_bounds__(256)
-    router_split_kernel(const float* __restrict__ Wr, size_t n, __nv_bfloat16* __restrict__ Wr3) {
+    router_split_kernel(const float* __restrict__ Wr, size_t n, __nv_bfloat16* __restrict__ Wr3,
+                        int* status) {
+  pdl_launch_dependents();
+  pdl_wait();
+  if (blockIdx.x == 0 && threadIdx.x == 0) {  // first kernel of a forward: clear the status
+    status[0] = 0;
+    status[1] = 0;
+  }
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x) {
     const float w = Wr[i];
@@ -86,6 +93,8 @@ __global__ void __launch_bounds__(R_THREADS, 1)
                        const __grid_constant__ CUtensorMap tmW3, int T, int E, int k_steps,
                        int S, float* __restrict__ partial, int* status,
                        unsigned long long timeout_ns) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -270,6 +279,8 @@ __global__ void __launch_bounds__(SEL_WARPS * 32)
                          RouterParams p, int32_t* __restrict__ topk_ids,
                          float* __restrict__ topk_w) {
   __shared__ float sc[SEL_WARPS * 2][RBN];  // bias-corrected scores of each token
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int half = lane >> 4, sl = lane & 15;
   const int T = p.T, E = p.E;
@@ -299,7 +310,7 @@ __global__ void __launch_bounds__(SEL_WARPS * 32)
         l = partial[(size_t)t * E + e];
         for (int k = 1; k < S; ++k) l += partial[((size_t)k * T + t) * E + e];
       }
-      s[i] = 1.0f / (1.0f + expf(-l));
+      s[i] = __frcp_rn(1.0f + expf(-l));  // correctly rounded: the same value as 1/(1+e^-l)
       c[i] = s[i] + b[i];
     }
     if (group_step) {
@@ -401,10 +412,12 @@ cudaError_t launch_router(const void* x, const float* Wr, const float* bias, con
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) +
                                             (((size_t)3 * E * H * 2 + 255) & ~(size_t)255));
   const size_t n = (size_t)E * H;
-  router_split_kernel<<<(int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, stream>>>(
-      Wr, n, Wr3);
+  const int split_grid = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+  cudaError_t err = launch_chained(router_split_kernel, dim3(split_grid), dim3(256), 0, stream, Wr,
+                                   n, Wr3, status);
+  if (err != cudaSuccess) return err;
   CUtensorMap tmX, tmW3;
-  cudaError_t err = make_tmap_2d(&tmX, x, (uint64_t)T, (uint64_t)H);
+  err = make_tmap_2d(&tmX, x, (uint64_t)T, (uint64_t)H);
   if (err != cudaSuccess) return err;
   err = make_tmap_3d(&tmW3, Wr3, 3, (uint64_t)E, (uint64_t)H);
   if (err != cudaSuccess) return err;
@@ -414,13 +427,15 @@ cudaError_t launch_router(const void* x, const float* Wr, const float* bias, con
   const int S = router_splits(H);
   const int items = ((T + RBM - 1) / RBM) * S;
   const int grid = items < num_sms() ? items : num_sms();
-  router_gemm_kernel<<<grid, R_THREADS, R_SMEM_BYTES, stream>>>(tmX, tmW3, T, E, H / RBK, S,
-                                                                 partial, status, timeout_ns);
+  err = launch_chained(router_gemm_kernel, dim3(grid), dim3(R_THREADS), R_SMEM_BYTES, stream, tmX,
+                       tmW3, T, E, H / RBK, S, partial, status, timeout_ns);
+  if (err != cudaSuccess) return err;
   int sel_grid = ((T + 1) / 2 + SEL_WARPS - 1) / SEL_WARPS;
   const int cap = num_sms() * 16;
   if (sel_grid > cap) sel_grid = cap;
-  router_select_kernel<<<sel_grid, SEL_WARPS * 32, 0, stream>>>(partial, S, bias, p, topk_ids,
-                                                                 topk_w);
+  err = launch_chained(router_select_kernel, dim3(sel_grid), dim3(SEL_WARPS * 32), 0, stream,
+                       (const float*)partial, S, bias, p, topk_ids, topk_w);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

@@ -198,23 +198,30 @@ def permute(topk_ids: torch.Tensor, cfg: BlockConfig, topk_w: Optional[torch.Ten
 
 
 class StageTimer:
-    """CUDA events recorded by moe_forward around each stage, on its stream."""
+    """CUDA events recorded by moe_forward around stages, on its stream.
 
-    def __init__(self):
-        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(NUM_STAGES + 1)]
+    ``stages`` selects the stages to time (default: all).  Every recorded
+    event serialises the kernels around it, so time only what is needed."""
+
+    def __init__(self, stages=STAGES):
+        idx = sorted({i for name in stages for i in (STAGES.index(name), STAGES.index(name) + 1)})
+        self.events = [torch.cuda.Event(enable_timing=True) if i in idx else None
+                       for i in range(NUM_STAGES + 1)]
         for e in self.events:  # torch creates the CUDA event on its first record
-            e.record()
-        handles = [e.cuda_event for e in self.events]
-        if not all(handles):
+            if e is not None:
+                e.record()
+        handles = [e.cuda_event if e is not None else None for e in self.events]
+        if not all(h for h, e in zip(handles, self.events) if e is not None):
             raise RuntimeError("could not create CUDA events for stage timing")
+        self.stages = tuple(stages)
         self._arr = (ctypes.c_void_p * (NUM_STAGES + 1))(*handles)
 
     def as_ptr(self):
         return ctypes.cast(self._arr, ctypes.POINTER(ctypes.c_void_p))
 
     def stage_ms(self):
-        return {STAGES[i]: self.events[i].elapsed_time(self.events[i + 1])
-                for i in range(NUM_STAGES)}
+        return {name: self.events[STAGES.index(name)].elapsed_time(
+                    self.events[STAGES.index(name) + 1]) for name in self.stages}
 
 
 def forward(x: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor, w13: torch.Tensor,
