@@ -191,6 +191,45 @@ MOE_API int32_t moe_forward(const void* x, const float* Wr, const float* bias, c
                     void* out, const moe_forward_opts_t* opts, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/* Workspace bytes of moe_forward_host: those of moe_forward plus four
+ * [T,H] bf16 staging buffers (two for inputs, two for outputs); 0 for an
+ * invalid configuration. */
+MOE_API size_t moe_forward_host_workspace_bytes(const moe_cfg_t* cfg);
+
+/* moe_forward over n_batches independent batches of cfg->T tokens that live
+ * in HOST memory: batch b is copied in from x_host[b], run through the block
+ * (the same kernels and bits as moe_forward, no residual) and copied out to
+ * out_host[b].  The sources define only the block itself; streaming
+ * host-resident batches through it, with the copies of the neighbouring
+ * batches overlapping each batch's kernels, is this library's own addition.
+ *   x_host, out_host  host arrays of n_batches host pointers, each to a
+ *                     [T,H] bf16 row-major batch; a pointer may repeat (the
+ *                     same input several times, one output buffer reused),
+ *                     but no output may overlap any input.
+ *                     Page-locked memory (cudaHostAlloc / cudaHostRegister)
+ *                     lets the copies overlap the kernels; pageable memory
+ *                     gives the same results with the copies serialised.
+ *   Wr ... ws2        device weights, as for moe_forward
+ *   workspace         device, moe_forward_host_workspace_bytes(cfg) bytes,
+ *                     256-byte aligned
+ *   stream            runs the kernels; h2d_stream / d2h_stream run the
+ *                     copies in / out (NULL: stream itself, no overlap).
+ * Everything starts after the work already queued on stream, and work queued
+ * on stream after this call starts only once every out_host[b] is written;
+ * the host buffers must stay valid until then.  Batches run in order; inputs
+ * are double-buffered so that batch b+1 is copied in while batch b computes
+ * and batch b-1 is copied out.  The status word is cleared by the first
+ * batch only, so moe_read_device_status reports the first device-side error
+ * of any batch.  Host checks (as moe_forward, plus n_batches < 0, a NULL
+ * batch pointer or an output overlapping an input) launch nothing; a CUDA
+ * failure part-way returns MOE_ERR_CUDA with the earlier batches queued. */
+MOE_API int32_t moe_forward_host(const void* const* x_host, void* const* out_host,
+                                 int32_t n_batches, const float* Wr, const float* bias,
+                                 const void* w13, const void* w2, const void* ws13,
+                                 const void* ws2, const moe_cfg_t* cfg, void* workspace,
+                                 size_t workspace_bytes, void* stream, void* h2d_stream,
+                                 void* d2h_stream);
+
 /* RMSNorm with fp32 accumulation ([S2]: RMSNorm accumulates in fp32), for a
  * residual stack of blocks: xn = bf16(x * rsqrt(mean(x^2) + eps) * gamma).
  *   x device bf16 [T,H]; gamma device fp32 [H] or NULL (= 1); xn device bf16 [T,H]. */

@@ -124,6 +124,7 @@ RouterParams router_params(const moe_cfg_t& c) {
   p.topk_group = c.topk_group;
   p.norm_topk_prob = c.norm_topk_prob;
   p.rsf = c.routed_scaling_factor;
+  p.clear_status = 1;
   return p;
 }
 
@@ -133,98 +134,24 @@ RouterParams router_params(const moe_cfg_t& c) {
     if (e_ != cudaSuccess) return MOE_ERR_CUDA; \
   } while (0)
 
-}  // namespace
-
-extern "C" {
-
-const char* moe_status_string(int32_t status) {
-  switch (status) {
-    case MOE_OK: return "MOE_OK";
-    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument or configuration";
-    case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE: shape outside the kernels' limits";
-    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, misaligned or too small";
-    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call failed";
-    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT: a device-side wait ran out";
-    case MOE_ERR_DEVICE_INDEX: return "MOE_ERR_DEVICE_INDEX: an expert id outside [0, E)";
-    case MOE_ERR_NO_DEVICE: return "MOE_ERR_NO_DEVICE: no usable CUDA device";
-    default: return "unknown moe_status_t";
-  }
-}
-
-int32_t moe_check_config(const moe_cfg_t* cfg) { return check_cfg(cfg); }
-
-size_t moe_route_workspace_bytes(const moe_cfg_t* cfg) {
-  if (check_cfg(cfg) != MOE_OK) return 0;
-  return align_up(sizeof(DevStatus)) + align_up(router_scratch_bytes(cfg->T, cfg->H, cfg->E));
-}
-
-size_t moe_permute_workspace_bytes(const moe_cfg_t* cfg) {
-  if (check_cfg(cfg) != MOE_OK) return 0;
-  return perm_layout(*cfg).total;
-}
-
-size_t moe_workspace_bytes(const moe_cfg_t* cfg) {
-  if (check_cfg(cfg) != MOE_OK) return 0;
-  return fwd_layout(*cfg).total;
-}
-
-int32_t moe_route(const void* x, const float* Wr, const float* bias, const moe_cfg_t* cfg,
-                  int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes,
-                  void* stream) {
-  const int32_t st = check_cfg(cfg);
-  if (st != MOE_OK) return st;
-  if (cfg->T == 0) return MOE_OK;
-  if (!x || !Wr || !bias || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
-  if (!ws_ok(workspace, workspace_bytes, moe_route_workspace_bytes(cfg))) return MOE_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int* status = at<int>(workspace, 0);
-  return cuda_status(launch_router(x, Wr, bias, router_params(*cfg), topk_ids, topk_w,
-                                   at<void>(workspace, align_up(sizeof(DevStatus))), status,
-                                   DEFAULT_TIMEOUT_NS, s));
-}
-
-int32_t moe_permute(const int32_t* topk_ids, const float* topk_w, const void* x,
-                    const moe_cfg_t* cfg, int32_t* expert_offsets, int32_t* row_of,
-                    int32_t* tok_of, float* w_of, void* xp, void* workspace,
-                    size_t workspace_bytes, void* stream) {
-  const int32_t st = check_cfg(cfg);
-  if (st != MOE_OK) return st;
-  if (cfg->T == 0) return MOE_OK;
-  if (!topk_ids || !expert_offsets || !row_of || !tok_of) return MOE_ERR_INVALID_ARG;
-  if (xp && !x) return MOE_ERR_INVALID_ARG;
-  const PermLayout L = perm_layout(*cfg);
-  if (!ws_ok(workspace, workspace_bytes, L.total)) return MOE_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int* status = at<int>(workspace, L.status);
-  RMOE_TRY(launch_status_reset(status, s));
-  PermuteOut o;
-  o.status = status;
-  o.blk_hist = at<int>(workspace, L.blk_hist);
-  o.expert_offsets = expert_offsets;
-  o.mtile_start = at<int>(workspace, L.mtiles);
-  o.row_of = row_of;
-  o.tok_of = tok_of;
-  o.w_of = w_of;
-  o.xp = xp;
-  return cuda_status(launch_permute(topk_ids, topk_w, x, cfg->T, cfg->H, cfg->E, cfg->top_k, o, s));
-}
-
-int32_t moe_forward(const void* x, const float* Wr, const float* bias, const void* w13,
-                    const void* w2, const void* ws13, const void* ws2, const moe_cfg_t* cfg,
-                    void* out, const moe_forward_opts_t* opts, void* workspace,
-                    size_t workspace_bytes, void* stream) {
-  const int32_t st = check_cfg(cfg);
-  if (st != MOE_OK) return st;
-  const moe_cfg_t& c = *cfg;
-  if (c.T == 0) return MOE_OK;
+// Host checks of moe_forward (the configuration already checked).
+int32_t check_forward_args(const moe_cfg_t& c, const void* x, const float* Wr, const float* bias,
+                           const void* w13, const void* w2, const void* ws13, const void* ws2,
+                           const void* out, const moe_forward_opts_t* opts) {
   if (!x || !Wr || !bias || !w13 || !w2 || !out) return MOE_ERR_INVALID_ARG;
   if ((c.I_shared > 0) != (ws13 != nullptr && ws2 != nullptr)) return MOE_ERR_INVALID_ARG;
   if (out == x) return MOE_ERR_INVALID_ARG;
-  const FwdLayout L = fwd_layout(c);
-  if (!ws_ok(workspace, workspace_bytes, L.total)) return MOE_ERR_WORKSPACE;
   if (opts && opts->wait_timeout_ns < 0) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
 
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+// The launch sequence of one block forward; arguments already checked, T > 0.
+// clear_status: the router's first kernel clears the status word.
+int32_t forward_impl(const void* x, const float* Wr, const float* bias, const void* w13,
+                     const void* w2, const void* ws13, const void* ws2, const moe_cfg_t& c,
+                     void* out, const moe_forward_opts_t* opts, void* workspace, bool clear_status,
+                     cudaStream_t s) {
+  const FwdLayout L = fwd_layout(c);
   void** ev = opts ? opts->stage_events : nullptr;
   const unsigned long long timeout =
       (opts && opts->wait_timeout_ns > 0) ? (unsigned long long)opts->wait_timeout_ns
@@ -268,8 +195,10 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
   };
 
   RMOE_TRY(record(MOE_STAGE_ROUTER));
-  RMOE_TRY(launch_router(x, Wr, bias, router_params(c), ids, tw, at<void>(workspace, L.router),
-                         status, timeout, s));
+  RouterParams rp = router_params(c);
+  rp.clear_status = clear_status ? 1 : 0;
+  RMOE_TRY(launch_router(x, Wr, bias, rp, ids, tw, at<void>(workspace, L.router), status, timeout,
+                         s));
 
   RMOE_TRY(record(MOE_STAGE_PERMUTE));
   PermuteOut o;
@@ -377,6 +306,172 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
   const void* residual = opts ? opts->residual : nullptr;
   RMOE_TRY(launch_combine_slots(Y, row_of, c.top_k, c.T, c.H, slots, residual, out, s));
   RMOE_TRY(record(MOE_NUM_STAGES));
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int32_t status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument or configuration";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE: shape outside the kernels' limits";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call failed";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT: a device-side wait ran out";
+    case MOE_ERR_DEVICE_INDEX: return "MOE_ERR_DEVICE_INDEX: an expert id outside [0, E)";
+    case MOE_ERR_NO_DEVICE: return "MOE_ERR_NO_DEVICE: no usable CUDA device";
+    default: return "unknown moe_status_t";
+  }
+}
+
+int32_t moe_check_config(const moe_cfg_t* cfg) { return check_cfg(cfg); }
+
+size_t moe_route_workspace_bytes(const moe_cfg_t* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return align_up(sizeof(DevStatus)) + align_up(router_scratch_bytes(cfg->T, cfg->H, cfg->E));
+}
+
+size_t moe_permute_workspace_bytes(const moe_cfg_t* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return perm_layout(*cfg).total;
+}
+
+size_t moe_workspace_bytes(const moe_cfg_t* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return fwd_layout(*cfg).total;
+}
+
+int32_t moe_route(const void* x, const float* Wr, const float* bias, const moe_cfg_t* cfg,
+                  int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  const int32_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !Wr || !bias || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!ws_ok(workspace, workspace_bytes, moe_route_workspace_bytes(cfg))) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = at<int>(workspace, 0);
+  return cuda_status(launch_router(x, Wr, bias, router_params(*cfg), topk_ids, topk_w,
+                                   at<void>(workspace, align_up(sizeof(DevStatus))), status,
+                                   DEFAULT_TIMEOUT_NS, s));
+}
+
+int32_t moe_permute(const int32_t* topk_ids, const float* topk_w, const void* x,
+                    const moe_cfg_t* cfg, int32_t* expert_offsets, int32_t* row_of,
+                    int32_t* tok_of, float* w_of, void* xp, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  const int32_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!topk_ids || !expert_offsets || !row_of || !tok_of) return MOE_ERR_INVALID_ARG;
+  if (xp && !x) return MOE_ERR_INVALID_ARG;
+  const PermLayout L = perm_layout(*cfg);
+  if (!ws_ok(workspace, workspace_bytes, L.total)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = at<int>(workspace, L.status);
+  RMOE_TRY(launch_status_reset(status, s));
+  PermuteOut o;
+  o.status = status;
+  o.blk_hist = at<int>(workspace, L.blk_hist);
+  o.expert_offsets = expert_offsets;
+  o.mtile_start = at<int>(workspace, L.mtiles);
+  o.row_of = row_of;
+  o.tok_of = tok_of;
+  o.w_of = w_of;
+  o.xp = xp;
+  return cuda_status(launch_permute(topk_ids, topk_w, x, cfg->T, cfg->H, cfg->E, cfg->top_k, o, s));
+}
+
+int32_t moe_forward(const void* x, const float* Wr, const float* bias, const void* w13,
+                    const void* w2, const void* ws13, const void* ws2, const moe_cfg_t* cfg,
+                    void* out, const moe_forward_opts_t* opts, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  const int32_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  const moe_cfg_t& c = *cfg;
+  if (c.T == 0) return MOE_OK;
+  const int32_t a = check_forward_args(c, x, Wr, bias, w13, w2, ws13, ws2, out, opts);
+  if (a != MOE_OK) return a;
+  if (!ws_ok(workspace, workspace_bytes, fwd_layout(c).total)) return MOE_ERR_WORKSPACE;
+  return forward_impl(x, Wr, bias, w13, w2, ws13, ws2, c, out, opts, workspace, true,
+                      static_cast<cudaStream_t>(stream));
+}
+
+size_t moe_forward_host_workspace_bytes(const moe_cfg_t* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return fwd_layout(*cfg).total + 4 * align_up((size_t)cfg->T * cfg->H * 2);
+}
+
+int32_t moe_forward_host(const void* const* x_host, void* const* out_host, int32_t n_batches,
+                         const float* Wr, const float* bias, const void* w13, const void* w2,
+                         const void* ws13, const void* ws2, const moe_cfg_t* cfg, void* workspace,
+                         size_t workspace_bytes, void* stream, void* h2d_stream,
+                         void* d2h_stream) {
+  const int32_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  const moe_cfg_t& c = *cfg;
+  if (n_batches < 0) return MOE_ERR_INVALID_ARG;
+  if (n_batches == 0 || c.T == 0) return MOE_OK;
+  if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  const size_t bytes = (size_t)c.T * c.H * 2;
+  for (int b = 0; b < n_batches; ++b) {
+    if (!x_host[b] || !out_host[b]) return MOE_ERR_INVALID_ARG;
+    // an output must not overlap any batch's input: later batches read theirs
+    // after earlier outputs have landed
+    const uintptr_t o0 = reinterpret_cast<uintptr_t>(out_host[b]);
+    for (int q = 0; q < n_batches; ++q) {
+      const uintptr_t x0 = reinterpret_cast<uintptr_t>(x_host[q]);
+      if (o0 < x0 + bytes && x0 < o0 + bytes) return MOE_ERR_INVALID_ARG;
+    }
+  }
+  const FwdLayout L = fwd_layout(c);
+  const size_t stage = align_up(bytes);
+  if (!ws_ok(workspace, workspace_bytes, L.total + 4 * stage)) return MOE_ERR_WORKSPACE;
+  // staging buffers after the forward's own workspace: x of batches b % 2,
+  // out of batches b % 2 (one batch computes while the next arrives and the
+  // previous one leaves)
+  void* xs[2] = {at<void>(workspace, L.total), at<void>(workspace, L.total + stage)};
+  void* os[2] = {at<void>(workspace, L.total + 2 * stage), at<void>(workspace, L.total + 3 * stage)};
+  const int32_t a = check_forward_args(c, xs[0], Wr, bias, w13, w2, ws13, ws2, os[0], nullptr);
+  if (a != MOE_OK) return a;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t hs = h2d_stream ? static_cast<cudaStream_t>(h2d_stream) : s;
+  cudaStream_t ds = d2h_stream ? static_cast<cudaStream_t>(d2h_stream) : s;
+  // events: start, and per staging slot: input landed, forward done, output read
+  struct Events {
+    cudaEvent_t e[7] = {};
+    ~Events() {  // released by the driver once the recorded work completes
+      for (cudaEvent_t x : e)
+        if (x) cudaEventDestroy(x);
+    }
+  } ev;
+  for (cudaEvent_t& e : ev.e) RMOE_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+  cudaEvent_t start = ev.e[0], x_in[2] = {ev.e[1], ev.e[2]}, done[2] = {ev.e[3], ev.e[4]},
+              o_out[2] = {ev.e[5], ev.e[6]};
+  RMOE_TRY(cudaEventRecord(start, s));  // after the work already queued on stream
+  RMOE_TRY(cudaStreamWaitEvent(hs, start, 0));
+  RMOE_TRY(cudaStreamWaitEvent(ds, start, 0));
+  for (int b = 0; b < n_batches; ++b) {
+    const int k = b & 1;
+    if (b >= 2) RMOE_TRY(cudaStreamWaitEvent(hs, done[k], 0));  // batch b-2 has read xs[k]
+    RMOE_TRY(cudaMemcpyAsync(xs[k], x_host[b], bytes, cudaMemcpyHostToDevice, hs));
+    RMOE_TRY(cudaEventRecord(x_in[k], hs));
+    RMOE_TRY(cudaStreamWaitEvent(s, x_in[k], 0));
+    if (b >= 2) RMOE_TRY(cudaStreamWaitEvent(s, o_out[k], 0));  // os[k] copied out
+    const int32_t r = forward_impl(xs[k], Wr, bias, w13, w2, ws13, ws2, c, os[k], nullptr,
+                                   workspace, b == 0, s);
+    if (r != MOE_OK) return r;
+    RMOE_TRY(cudaEventRecord(done[k], s));
+    RMOE_TRY(cudaStreamWaitEvent(ds, done[k], 0));
+    RMOE_TRY(cudaMemcpyAsync(out_host[b], os[k], bytes, cudaMemcpyDeviceToHost, ds));
+    RMOE_TRY(cudaEventRecord(o_out[k], ds));
+  }
+  // the copies out run in order on one stream: the last one covers them all
+  RMOE_TRY(cudaStreamWaitEvent(s, o_out[(n_batches - 1) & 1], 0));
   return MOE_OK;
 }
 

@@ -31,13 +31,14 @@ cudaError_t launch_chained(void (*k)(KArgs...), dim3 grid, dim3 block, size_t sm
 struct RouterParams {
   int T, H, E, top_k, n_group, topk_group, norm_topk_prob;
   float rsf;
+  int clear_status;  // 1: the router's first kernel clears the status word
 };
 
 // Router on the tensor cores: scratch holds the 3-term bf16 split of Wr and the
 // fp32 partial logits of the K chunks (router_scratch_bytes).
 int router_splits(int H);
 size_t router_scratch_bytes(int T, int H, int E);
-// Also clears the status word (the first kernel of a forward).
+// Also clears the status word when p.clear_status is set (the first kernel of a forward).
 cudaError_t launch_router(const void* x, const float* Wr, const float* bias, const RouterParams& p,
                           int32_t* topk_ids, float* topk_w, void* scratch, int* status,
                           unsigned long long timeout_ns, cudaStream_t stream);

@@ -64,10 +64,10 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, uint6
 
 __global__ void __launch_bounds__(256)
     router_split_kernel(const float* __restrict__ Wr, size_t n, __nv_bfloat16* __restrict__ Wr3,
-                        int* status) {
+                        int* status, int clear_status) {
   pdl_launch_dependents();
   pdl_wait();
-  if (blockIdx.x == 0 && threadIdx.x == 0) {  // first kernel of a forward: clear the status
+  if (clear_status && blockIdx.x == 0 && threadIdx.x == 0) {  // first kernel of a forward
     status[0] = 0;
     status[1] = 0;
   }
@@ -414,7 +414,7 @@ cudaError_t launch_router(const void* x, const float* Wr, const float* bias, con
   const size_t n = (size_t)E * H;
   const int split_grid = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
   cudaError_t err = launch_chained(router_split_kernel, dim3(split_grid), dim3(256), 0, stream, Wr,
-                                   n, Wr3, status);
+                                   n, Wr3, status, p.clear_status);
   if (err != cudaSuccess) return err;
   CUtensorMap tmX, tmW3;
   err = make_tmap_2d(&tmX, x, (uint64_t)T, (uint64_t)H);

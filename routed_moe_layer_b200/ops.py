@@ -94,6 +94,9 @@ def lib() -> ctypes.CDLL:
         "moe_permute": (i32, [vp, vp, vp, cfgp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "moe_forward": (i32, [vp, vp, vp, vp, vp, vp, vp, cfgp, vp,
                               ctypes.POINTER(MoeForwardOpts), vp, sz, vp]),
+        "moe_forward_host_workspace_bytes": (sz, [cfgp]),
+        "moe_forward_host": (i32, [ctypes.POINTER(vp), ctypes.POINTER(vp), i32, vp, vp, vp, vp,
+                                   vp, vp, cfgp, vp, sz, vp, vp, vp]),
         "moe_rmsnorm": (i32, [vp, vp, ctypes.c_float, i32, i32, vp, vp]),
         "moe_read_device_status": (i32, [vp, ctypes.POINTER(i32), vp]),
         "moe_selftest_wait_timeout": (i32, [vp, i64, vp]),
@@ -263,6 +266,65 @@ def forward(x: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor, w13: torch.Te
                              _ptr(ws2), ctypes.byref(c), _ptr(out), ctypes.byref(opts),
                              _ptr(workspace), workspace.numel(), _stream_ptr()), "moe_forward")
     return out
+
+
+def forward_host_workspace_bytes(cfg: BlockConfig) -> int:
+    c = cfg.c()
+    return int(lib().moe_forward_host_workspace_bytes(ctypes.byref(c)))
+
+
+def _need_host(t: torch.Tensor, name: str, shape: Sequence[int]):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be torch.bfloat16, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def forward_host(x_host: Sequence[torch.Tensor], out_host: Sequence[torch.Tensor],
+                 Wr: torch.Tensor, bias: torch.Tensor, w13: torch.Tensor, w2: torch.Tensor,
+                 ws13: Optional[torch.Tensor], ws2: Optional[torch.Tensor], cfg: BlockConfig,
+                 workspace: Optional[torch.Tensor] = None,
+                 copy_streams: Optional[Sequence[torch.cuda.Stream]] = None):
+    """Block forward over host-resident batches (moe_forward_host).
+
+    x_host[b] / out_host[b]: CPU bf16 [T,H] tensors (pin them for overlap).
+    Kernels run on the current stream; copy_streams = (h2d, d2h) run the copies
+    (None: the current stream, no overlap).  Returns once queued: synchronise
+    the current stream before reading out_host."""
+    n = len(x_host)
+    if len(out_host) != n:
+        raise ValueError("x_host and out_host must have the same length")
+    T, H, E, I, Is = cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared
+    for b in range(n):
+        _need_host(x_host[b], f"x_host[{b}]", (T, H))
+        _need_host(out_host[b], f"out_host[{b}]", (T, H))
+    _need(Wr, "Wr", torch.float32, (E, H))
+    _need(bias, "bias", torch.float32, (E,))
+    _need(w13, "w13", torch.bfloat16, (E, 2 * I, H))
+    _need(w2, "w2", torch.bfloat16, (E, H, I))
+    if Is > 0:
+        _need(ws13, "ws13", torch.bfloat16, (2 * Is, H))
+        _need(ws2, "ws2", torch.bfloat16, (H, Is))
+    if workspace is None:
+        workspace = alloc_workspace(forward_host_workspace_bytes(cfg), Wr.device)
+    xs = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in x_host])
+    os_ = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in out_host])
+    h2d = d2h = None
+    if copy_streams is not None:
+        h2d = ctypes.c_void_p(copy_streams[0].cuda_stream)
+        d2h = ctypes.c_void_p(copy_streams[1].cuda_stream)
+    c = cfg.c()
+    _check(lib().moe_forward_host(xs, os_, n, _ptr(Wr), _ptr(bias), _ptr(w13), _ptr(w2),
+                                  _ptr(ws13), _ptr(ws2), ctypes.byref(c), _ptr(workspace),
+                                  workspace.numel(), _stream_ptr(), h2d, d2h),
+           "moe_forward_host")
+    return workspace
 
 
 def rmsnorm(x: torch.Tensor, gamma: Optional[torch.Tensor] = None, eps: float = 1e-6,

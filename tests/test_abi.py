@@ -143,3 +143,31 @@ def test_route_permute_rmsnorm_reject_bad_arguments(L):
     assert L.moe_rmsnorm(FAKE, None, ctypes.c_float(1e-6), 4, 100, FAKE, None) == 1
     assert L.moe_rmsnorm(FAKE, None, ctypes.c_float(-1.0), 4, 128, FAKE, None) == 1
     assert L.moe_selftest_wait_timeout(FAKE, 0, None) == 1
+
+
+def test_forward_host_rejects_bad_arguments_on_the_host(L):
+    c = BlockConfig(T=64, H=256, I=128, I_shared=128).c()
+    need = L.moe_forward_host_workspace_bytes(ctypes.byref(c))
+    assert need == L.moe_workspace_bytes(ctypes.byref(c)) + 4 * 64 * 256 * 2
+    P = ctypes.c_void_p * 2
+    xs = P(0x100000, 0x100000)          # one input buffer used twice: allowed
+    outs = P(0x200000, 0x200000)        # one output buffer reused: allowed
+    w = [FAKE] * 6
+
+    def call(x, o, n, cfg=c, ws=FAKE, nbytes=need, weights=w):
+        return L.moe_forward_host(x, o, n, *weights, ctypes.byref(cfg), ws, nbytes, None, None,
+                                  None)
+
+    assert call(xs, outs, -1) == 1
+    assert call(None, outs, 2) == 1
+    assert call(xs, None, 2) == 1
+    assert call(P(0x100000, 0), outs, 2) == 1                   # NULL batch pointer
+    assert call(xs, P(0x200000, 0x100000 + 64 * 256), 2) == 1  # out overlaps an input's tail
+    assert call(xs, outs, 2, nbytes=need - 1) == 3
+    assert call(xs, outs, 2, ws=ctypes.c_void_p(0x10010)) == 3
+    assert call(xs, outs, 2, weights=[FAKE] * 4 + [None, None]) == 1  # shared weights missing
+    assert call(xs, outs, 2, cfg=BlockConfig(T=64, H=250).c()) == 2
+    # nothing to do: no batches, or T = 0
+    assert call(None, None, 0) == 0
+    z = BlockConfig(T=0, H=256, I=128, I_shared=128).c()
+    assert call(None, None, 3, cfg=z) == 0

@@ -229,6 +229,37 @@ def test_forward_deterministic_and_isolated():
         assert torch.equal(p, a[lo:hi])
 
 
+@pytest.mark.parametrize("overlap", [True, False])
+def test_forward_host_batches_match_device_forward(overlap):
+    """Host-resident batches streamed through the block give, bit for bit, the
+    device entry point's output for each batch (and the oracle's, to tolerance)."""
+    T, H = 700, 512
+    cfg = BlockConfig(T=T, H=H, I=256, I_shared=256)
+    d = inputs.make_block_inputs(T, H, seed=21, I=256, I_shared=256, unit_scale=True)
+    dd = _dev(d)
+    n = 5
+    g = torch.Generator().manual_seed(77)
+    xs = [torch.randn((T, H), generator=g).to(torch.bfloat16) for _ in range(n - 1)]
+    xs.append(xs[0])  # a repeated input pointer is allowed
+    if overlap:
+        xs = [x.pin_memory() for x in xs]
+    outs = [torch.zeros((T, H), dtype=torch.bfloat16) for _ in range(n)]
+    if overlap:
+        outs = [o.pin_memory() for o in outs]
+    streams = (torch.cuda.Stream(), torch.cuda.Stream()) if overlap else None
+    ws = ops.forward_host(xs, outs, dd["Wr"], dd["bias"], dd["w13"], dd["w2"], dd["ws13"],
+                          dd["ws2"], cfg, copy_streams=streams)
+    torch.cuda.current_stream().synchronize()
+    code, site = ops.read_device_status(ws)
+    assert code == 0, (ops.status_string(code), site)
+    for b in range(n):
+        ref, _, _ = _run(dict(dd, x=xs[b].to(DEV)), cfg)
+        assert torch.equal(outs[b], ref.cpu()), b
+    ids_b = _run(dict(dd, x=xs[1].to(DEV)), cfg)[1]
+    d_np = {k: parity.to_np(v) for k, v in dict(d, x=xs[1]).items() if v is not None}
+    parity.check_output(outs[1], ids_b, d_np, cfg)
+
+
 # ------------------------------------------------------------------ RMSNorm, residual stack
 def test_rmsnorm_matches_oracle():
     T, H = 333, 2048
