@@ -45,6 +45,7 @@ cudaError_t launch_router(const void* x, const float* Wr, const float* bias, con
 
 // ------------------------------------------------------------------ permute
 constexpr int PERMUTE_TOK = 256;  // tokens per counting block
+constexpr int PERMUTE_SMALL_T = 1024;  // single-CTA permutation up to this many tokens
 constexpr int MTILE = 256;        // rows per grouped-GEMM tile (one CTA-pair MMA)
 
 struct PermuteOut {

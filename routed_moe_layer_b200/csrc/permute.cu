@@ -13,6 +13,8 @@
 //               also the token-major slot position of every row.
 //   4. gather:  xp[row] = x[tok_of[row]], walking tokens in order so that each
 //               token row is read once (skipped when x is not given).
+// Up to PERMUTE_SMALL_T tokens, steps 1-3 run in one CTA (one token per
+// thread), which saves two launches on small batches.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -23,6 +25,7 @@ namespace {
 constexpr int PT = PERMUTE_TOK;      // tokens per block (8 warps)
 constexpr int PW = PERMUTE_TOK / 32; // warps per block
 constexpr int MAXE = 128;
+constexpr int MAX_TOPK_PERMUTE = 16;
 
 __device__ __forceinline__ void build_masks(const int32_t* __restrict__ ids, int T, int E,
                                             int top_k, uint32_t (*masks)[MAXE], int* status) {
@@ -57,11 +60,71 @@ __global__ void __launch_bounds__(PT)
   }
 }
 
+// Warp 0 of a CTA: exclusive prefixes over experts of the row counts tot[e]
+// and of their MTILE-row tiles, into excl_rows / excl_tiles [E+1] (shared).
+__device__ __forceinline__ void scan_experts_warp(const int* tot_of, int E, int* excl_rows,
+                                                  int* excl_tiles) {
+  const int lane = threadIdx.x & 31;
+  int loc_rows[MAXE / 32], loc_tiles[MAXE / 32];
+  int sr = 0, st = 0;
+#pragma unroll
+  for (int q = 0; q < MAXE / 32; ++q) {
+    const int ee = lane * (MAXE / 32) + q;
+    const int tot = ee < E ? tot_of[ee] : 0;
+    loc_rows[q] = tot;
+    loc_tiles[q] = (tot + MTILE - 1) / MTILE;
+    sr += loc_rows[q];
+    st += loc_tiles[q];
+  }
+  int ir = sr, it = st;  // inclusive warp scan of the per-lane sums
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, ir, off);
+    const int b = __shfl_up_sync(0xffffffffu, it, off);
+    if (lane >= off) {
+      ir += a;
+      it += b;
+    }
+  }
+  int run_r = ir - sr, run_t = it - st;
+#pragma unroll
+  for (int q = 0; q < MAXE / 32; ++q) {
+    const int ee = lane * (MAXE / 32) + q;
+    if (ee < E) {
+      excl_rows[ee] = run_r;
+      excl_tiles[ee] = run_t;
+    }
+    run_r += loc_rows[q];
+    run_t += loc_tiles[q];
+  }
+  if (lane == 31) {
+    excl_rows[E] = ir;
+    excl_tiles[E] = it;
+  }
+}
+
+// Writes the per-expert row offsets and tile prefixes ([E+1], plus group E+1
+// when extra_rows > 0) from the shared exclusive prefixes; threads 0..E.
+__device__ __forceinline__ void write_offsets(const int* excl_rows, const int* excl_tiles, int E,
+                                              int extra_rows, int* expert_offsets,
+                                              int* mtile_start) {
+  const int tid = threadIdx.x;
+  if (tid <= E) {
+    expert_offsets[tid] = excl_rows[tid];
+    if (mtile_start) mtile_start[tid] = excl_tiles[tid];
+  }
+  if (tid == 0 && extra_rows > 0) {  // one more group after the experts
+    expert_offsets[E + 1] = excl_rows[E] + extra_rows;
+    if (mtile_start) mtile_start[E + 1] = excl_tiles[E] + (extra_rows + MTILE - 1) / MTILE;
+  }
+}
+
 // One CTA of 1024 threads: expert e = tid % E, chunk ch = tid / E of the blocks.
 __global__ void __launch_bounds__(1024)
     permute_scan_kernel(int* __restrict__ blk_hist, int nblk, int E, int extra_rows,
                         int* __restrict__ expert_offsets, int* __restrict__ mtile_start) {
   __shared__ int part[1024];
+  __shared__ int tot[MAXE];
   __shared__ int excl_rows[MAXE + 1];
   __shared__ int excl_tiles[MAXE + 1];
   pdl_launch_dependents();
@@ -79,61 +142,19 @@ __global__ void __launch_bounds__(1024)
     part[ch * E + e] = s;
   }
   __syncthreads();
-  if (tid < 32) {
-    // warp 0: per-expert totals, chunk prefixes, then an exclusive scan over experts
-    int loc_rows[MAXE / 32], loc_tiles[MAXE / 32];
-    int sr = 0, st = 0;
-#pragma unroll
-    for (int q = 0; q < MAXE / 32; ++q) {
-      const int ee = tid * (MAXE / 32) + q;
-      int tot = 0;
-      if (ee < E) {
-        for (int c = 0; c < C; ++c) {
-          const int v = part[c * E + ee];
-          part[c * E + ee] = tot;  // exclusive prefix over chunks
-          tot += v;
-        }
-      }
-      loc_rows[q] = tot;
-      loc_tiles[q] = (tot + MTILE - 1) / MTILE;
-      sr += loc_rows[q];
-      st += loc_tiles[q];
+  if (tid < E) {  // per-expert total; chunk sums become exclusive prefixes over chunks
+    int run = 0;
+    for (int c = 0; c < C; ++c) {
+      const int v = part[c * E + tid];
+      part[c * E + tid] = run;
+      run += v;
     }
-    int ir = sr, it = st;  // inclusive warp scan of the per-lane sums
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int a = __shfl_up_sync(0xffffffffu, ir, off);
-      const int b = __shfl_up_sync(0xffffffffu, it, off);
-      if (tid >= off) {
-        ir += a;
-        it += b;
-      }
-    }
-    int run_r = ir - sr, run_t = it - st;
-#pragma unroll
-    for (int q = 0; q < MAXE / 32; ++q) {
-      const int ee = tid * (MAXE / 32) + q;
-      if (ee < E) {
-        excl_rows[ee] = run_r;
-        excl_tiles[ee] = run_t;
-      }
-      run_r += loc_rows[q];
-      run_t += loc_tiles[q];
-    }
-    if (tid == 31) {
-      excl_rows[E] = ir;
-      excl_tiles[E] = it;
-    }
+    tot[tid] = run;
   }
   __syncthreads();
-  if (tid <= E) {
-    expert_offsets[tid] = excl_rows[tid];
-    if (mtile_start) mtile_start[tid] = excl_tiles[tid];
-  }
-  if (tid == 0 && extra_rows > 0) {  // one more group after the experts
-    expert_offsets[E + 1] = excl_rows[E] + extra_rows;
-    if (mtile_start) mtile_start[E + 1] = excl_tiles[E] + (extra_rows + MTILE - 1) / MTILE;
-  }
+  if (tid < 32) scan_experts_warp(tot, E, excl_rows, excl_tiles);
+  __syncthreads();
+  write_offsets(excl_rows, excl_tiles, E, extra_rows, expert_offsets, mtile_start);
   if (active) {
     int run = excl_rows[e] + part[ch * E + e];
     for (int b = b0; b < b1; ++b) {
@@ -142,6 +163,71 @@ __global__ void __launch_bounds__(1024)
       blk_hist[i] = run;  // base row of expert e inside block b
       run += v;
     }
+  }
+}
+
+// T <= PERMUTE_SMALL_T: count, scan and scatter in one CTA of 1024 threads
+// (one token per thread); the same rows as the three-kernel path.
+__global__ void __launch_bounds__(1024)
+    permute_small_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T,
+                         int E, int top_k, int extra_rows, int* __restrict__ expert_offsets,
+                         int* __restrict__ mtile_start, int* __restrict__ row_of,
+                         int* __restrict__ tok_of, float* __restrict__ w_of,
+                         int* __restrict__ pos_of, int slot_stride, int* status) {
+  __shared__ uint32_t masks[32][MAXE];
+  __shared__ int wbase[32][MAXE];
+  __shared__ int tot[MAXE];
+  __shared__ int excl_rows[MAXE + 1];
+  __shared__ int excl_tiles[MAXE + 1];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < 32 * MAXE; i += 1024) (&masks[0][0])[i] = 0u;
+  __syncthreads();
+  const int t = tid;
+  int my_e[MAX_TOPK_PERMUTE];
+#pragma unroll
+  for (int j = 0; j < MAX_TOPK_PERMUTE; ++j) {
+    my_e[j] = -1;
+    if (t < T && j < top_k) {
+      const int e = ids[(size_t)t * top_k + j];
+      if (e >= 0 && e < E) {
+        my_e[j] = e;
+        atomicOr(&masks[warp][e], 1u << lane);
+      } else {
+        report_error(status, MOE_ERR_DEVICE_INDEX, 1);
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < E) {  // rows of expert e before each warp, and in total
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      wbase[w][tid] = run;
+      run += __popc(masks[w][tid]);
+    }
+    tot[tid] = run;
+  }
+  __syncthreads();
+  if (tid < 32) scan_experts_warp(tot, E, excl_rows, excl_tiles);
+  __syncthreads();
+  write_offsets(excl_rows, excl_tiles, E, extra_rows, expert_offsets, mtile_start);
+  if (t >= T) return;
+  const uint32_t lower = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < MAX_TOPK_PERMUTE; ++j) {
+    if (j >= top_k) break;
+    const size_t tj = (size_t)t * top_k + j;
+    const int e = my_e[j];
+    if (e < 0) {
+      row_of[tj] = -1;
+      continue;
+    }
+    const int row = excl_rows[e] + wbase[warp][e] + __popc(masks[warp][e] & lower);
+    row_of[tj] = row;
+    tok_of[row] = t;
+    if (w_of) w_of[row] = topk_w ? topk_w[tj] : 1.0f;
+    if (pos_of) pos_of[row] = t * slot_stride + j;
   }
 }
 
@@ -206,12 +292,34 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+cudaError_t launch_gather(const void* x, int T, int H, int top_k, const PermuteOut& o,
+                          cudaStream_t stream) {
+  if (o.xp && x) {
+    int grid = (T + 7) / 8;
+    const int cap = num_sms() * 8;
+    if (grid > cap) grid = cap;
+    const cudaError_t err = launch_chained(
+        gather_tokens_kernel, dim3(grid), dim3(256), 0, stream, static_cast<const __nv_bfloat16*>(x),
+        (const int*)o.row_of, T, H, top_k, static_cast<__nv_bfloat16*>(o.xp));
+    if (err != cudaSuccess) return err;
+  }
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const void* x, int T,
                            int H, int E, int top_k, const PermuteOut& o, cudaStream_t stream) {
+  cudaError_t err;
+  if (T <= PERMUTE_SMALL_T) {
+    err = launch_chained(permute_small_kernel, dim3(1), dim3(1024), 0, stream, topk_ids, topk_w, T,
+                         E, top_k, o.extra_rows, o.expert_offsets, o.mtile_start, o.row_of,
+                         o.tok_of, o.w_of, o.pos_of, o.slot_stride, o.status);
+    if (err != cudaSuccess) return err;
+    return launch_gather(x, T, H, top_k, o, stream);
+  }
   const int nblk = (T + PT - 1) / PT;
-  cudaError_t err = launch_chained(permute_count_kernel, dim3(nblk), dim3(PT), 0, stream, topk_ids,
+  err = launch_chained(permute_count_kernel, dim3(nblk), dim3(PT), 0, stream, topk_ids,
                                    T, E, top_k, o.blk_hist, o.status);
   if (err != cudaSuccess) return err;
   err = launch_chained(permute_scan_kernel, dim3(1), dim3(1024), 0, stream, o.blk_hist, nblk, E,
@@ -221,16 +329,7 @@ cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const v
                        T, E, top_k, (const int*)o.blk_hist, o.row_of, o.tok_of, o.w_of, o.pos_of,
                        o.slot_stride, o.status);
   if (err != cudaSuccess) return err;
-  if (o.xp && x) {
-    int grid = (T + 7) / 8;
-    const int cap = num_sms() * 8;
-    if (grid > cap) grid = cap;
-    err = launch_chained(gather_tokens_kernel, dim3(grid), dim3(256), 0, stream,
-                         static_cast<const __nv_bfloat16*>(x), (const int*)o.row_of, T, H, top_k,
-                         static_cast<__nv_bfloat16*>(o.xp));
-    if (err != cudaSuccess) return err;
-  }
-  return cudaGetLastError();
+  return launch_gather(x, T, H, top_k, o, stream);
 }
 
 }  // namespace rmoe

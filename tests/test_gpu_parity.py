@@ -84,8 +84,10 @@ def test_router_bias_forces_selection_not_weights():
 
 
 # ------------------------------------------------------------------ permutation
+# T <= 1024 runs the single-CTA path, larger T the three-kernel path
 @pytest.mark.parametrize("T,E,k", [(1, 8, 2), (255, 128, 8), (256, 128, 8), (257, 128, 8),
-                                   (1000, 16, 4), (19412, 128, 8)])
+                                   (1000, 16, 4), (1024, 128, 8), (1025, 128, 8), (3000, 64, 6),
+                                   (19412, 128, 8)])
 def test_permute_bit_exact(T, E, k):
     g = torch.Generator().manual_seed(T * 7 + E)
     ids = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
@@ -105,8 +107,9 @@ def test_permute_bit_exact(T, E, k):
     assert torch.equal(r["xp"].cpu(), x[torch.as_tensor(tok_of)])
 
 
-def test_permute_reports_bad_expert_id():
-    T, E, k = 64, 16, 2
+@pytest.mark.parametrize("T", [64, 2000])
+def test_permute_reports_bad_expert_id(T):
+    E, k = 16, 2
     ids = torch.tensor([[i % E, (i + 1) % E] for i in range(T)], dtype=torch.int32)
     ids[5, 1] = E  # out of range: skipped and reported
     cfg = BlockConfig(T=T, H=64, E=E, top_k=k, n_group=1, topk_group=1)
