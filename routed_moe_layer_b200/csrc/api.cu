@@ -61,6 +61,11 @@ int slots_per_token(const moe_cfg_t& c) { return c.top_k + (c.I_shared > 0 ? 1 :
 // come from x and its weights from ws13 / ws2.
 bool fuse_shared(const moe_cfg_t& c) { return c.I_shared > 0 && c.I_shared == c.I; }
 
+// Few rows per expert (at most 64 on average): the grouped GEMMs run with
+// swapped operands (weight rows on the MMA's M, the expert's rows on N), so
+// that tiles are not padded to 256 rows.  Decided from the shapes only.
+bool use_swap(const moe_cfg_t& c) { return (int64_t)c.T * c.top_k <= 64LL * c.E; }
+
 FwdLayout fwd_layout(const moe_cfg_t& c) {
   FwdLayout L;
   const size_t T = c.T, R = T * c.top_k, E = c.E;
@@ -145,6 +150,116 @@ int32_t check_forward_args(const moe_cfg_t& c, const void* x, const float* Wr, c
   return MOE_OK;
 }
 
+// The expert and shared-expert GEMMs with swapped operands (use_swap).
+template <typename Rec>
+cudaError_t swap_gemms(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp, __nv_bfloat16* h,
+                       __nv_bfloat16* hs, __nv_bfloat16* Y, const CUtensorMap& tm_w13,
+                       const CUtensorMap& tm_w2, const CUtensorMap& tm_ws13,
+                       const CUtensorMap& tm_ws2, const int* offsets, const PermuteOut& o,
+                       const GemmArgs& a, int sms, Rec& record, cudaStream_t s) {
+  const size_t T = c.T, R = T * c.top_k;
+  const int slots = slots_per_token(c);
+  const bool fused = fuse_shared(c);
+  const int groups = c.E + (fused ? 1 : 0);
+  const long long chunk_bound = (long long)(R / 128) + groups + 1;
+  CUtensorMap tm_xp, tm_x, tm_h, tm_h_shared, tm_hs;
+  cudaError_t e;
+  if ((e = make_tmap_2d_box(&tm_xp, xp, R, c.H, 32)) != cudaSuccess) return e;
+  if ((e = make_tmap_2d_box(&tm_h, h, R, c.I, 32)) != cudaSuccess) return e;
+  tm_x = tm_h_shared = tm_hs = tm_xp;  // unused unless there is a shared expert
+  if (c.I_shared > 0) {
+    if ((e = make_tmap_2d_box(&tm_x, x, T, c.H, 32)) != cudaSuccess) return e;
+    if (fused) {
+      if ((e = make_tmap_2d_box(&tm_h_shared, h + R * c.I, T, c.I, 32)) != cudaSuccess) return e;
+    } else {
+      if ((e = make_tmap_2d_box(&tm_hs, hs, T, c.I_shared, 32)) != cudaSuccess) return e;
+    }
+  }
+  if ((e = record(MOE_STAGE_EXPERT_UP)) != cudaSuccess) return e;
+  {  // h[r, i] = silu(W13g[i] . x_r) * (W13u[i] . x_r) per group (shared expert: group E)
+    GemmArgs g = a;
+    g.mtile_start = o.mtile_start;
+    g.row_start = offsets;
+    g.num_groups = groups;
+    if (fused) {
+      g.alt_group = c.E;
+      g.alt_row0 = (int)R;
+    }
+    g.n_tiles = (c.I + 127) / 128;
+    g.k_steps = c.H / 64;
+    g.n_out_tile = 128;
+    g.b_second = c.I;
+    g.out = h;
+    g.ldo = c.I;
+    g.n_valid = c.I;
+    const int grid = (int)std::min<long long>(sms, chunk_bound * g.n_tiles);
+    if ((e = launch_grouped_gemm_swap(EPI_SWIGLU, tm_w13, tm_xp, tm_ws13, tm_x, g, grid, s)) !=
+        cudaSuccess)
+      return e;
+  }
+  if ((e = record(MOE_STAGE_EXPERT_DOWN)) != cudaSuccess) return e;
+  {  // Y[pos_r, n] = w_r * (W2[n] . h_r) per expert; shared rows to slot top_k, unscaled
+    GemmArgs g = a;
+    g.mtile_start = o.mtile_start;
+    g.row_start = offsets;
+    g.num_groups = groups;
+    if (fused) {
+      g.alt_group = c.E;
+      g.alt_row0 = (int)R;
+    }
+    g.n_tiles = (c.H + 127) / 128;
+    g.k_steps = c.I / 64;
+    g.n_out_tile = 128;
+    g.out = Y;
+    g.ldo = c.H;
+    g.n_valid = c.H;
+    g.row_scale = o.w_of;
+    g.dest_pos = o.pos_of;
+    g.dest_mul = slots;
+    g.dest_add = c.top_k;
+    const int grid = (int)std::min<long long>(sms, chunk_bound * g.n_tiles);
+    if ((e = launch_grouped_gemm_swap(EPI_ROWSCALE, tm_w2, tm_h, tm_ws2, tm_h_shared, g, grid,
+                                      s)) != cudaSuccess)
+      return e;
+  }
+  if ((e = record(MOE_STAGE_SHARED_EXPERT)) != cudaSuccess) return e;
+  if (c.I_shared > 0 && !fused) {
+    const long long chunks = (long long)(T + 127) / 128;
+    {  // hs = silu(x . Ws13g^T) * (x . Ws13u^T)
+      GemmArgs g = a;
+      g.single_rows = c.T;
+      g.n_tiles = (c.I_shared + 127) / 128;
+      g.k_steps = c.H / 64;
+      g.n_out_tile = 128;
+      g.b_second = c.I_shared;
+      g.out = hs;
+      g.ldo = c.I_shared;
+      g.n_valid = c.I_shared;
+      const int grid = (int)std::min<long long>(sms, chunks * g.n_tiles);
+      if ((e = launch_grouped_gemm_swap(EPI_SWIGLU, tm_ws13, tm_x, tm_ws13, tm_x, g, grid, s)) !=
+          cudaSuccess)
+        return e;
+    }
+    {  // Y[t*slots + top_k] = hs . Ws2^T  (unscaled)
+      GemmArgs g = a;
+      g.single_rows = c.T;
+      g.n_tiles = (c.H + 127) / 128;
+      g.k_steps = c.I_shared / 64;
+      g.n_out_tile = 128;
+      g.out = Y;
+      g.ldo = c.H;
+      g.n_valid = c.H;
+      g.dest_mul = slots;
+      g.dest_add = c.top_k;
+      const int grid = (int)std::min<long long>(sms, chunks * g.n_tiles);
+      if ((e = launch_grouped_gemm_swap(EPI_ROWSCALE, tm_ws2, tm_hs, tm_ws2, tm_hs, g, grid, s)) !=
+          cudaSuccess)
+        return e;
+    }
+  }
+  return cudaSuccess;
+}
+
 // The launch sequence of one block forward; arguments already checked, T > 0.
 // clear_status: the router's first kernel clears the status word.
 int32_t forward_impl(const void* x, const float* Wr, const float* bias, const void* w13,
@@ -225,81 +340,86 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
   a.timeout_ns = timeout;
   a.alt_group = -1;
 
-  RMOE_TRY(record(MOE_STAGE_EXPERT_UP));
-  {  // h = silu(A . W13g^T) * (A . W13u^T) per group: A = gathered rows (experts), x (shared)
-    GemmArgs g = a;
-    g.mtile_start = mtiles;
-    g.row_start = offsets;
-    g.num_groups = groups;
-    if (fused) {
-      g.alt_group = c.E;
-      g.alt_row0 = (int)R;
-    }
-    g.n_tiles = (c.I + 127) / 128;
-    g.k_steps = c.H / 64;
-    g.n_out_tile = 128;
-    g.b_second = c.I;
-    g.out = h;
-    g.ldo = c.I;
-    g.n_valid = c.I;
-    const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
-    RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_xp, tm_w13, tm_x, tm_ws13, g, grid, s));
-  }
-  RMOE_TRY(record(MOE_STAGE_EXPERT_DOWN));
-  {  // Y[t*slots + j] = w_tj * (h . W2^T) per expert; shared rows to slot top_k, unscaled
-    GemmArgs g = a;
-    g.mtile_start = mtiles;
-    g.row_start = offsets;
-    g.num_groups = groups;
-    if (fused) {
-      g.alt_group = c.E;
-      g.alt_row0 = (int)R;
-    }
-    g.n_tiles = (c.H + 255) / 256;
-    g.k_steps = c.I / 64;
-    g.n_out_tile = 256;
-    g.b_second = 128;
-    g.out = Y;
-    g.ldo = c.H;
-    g.n_valid = c.H;
-    g.row_scale = o.w_of;
-    g.dest_pos = o.pos_of;
-    g.dest_mul = slots;
-    g.dest_add = c.top_k;
-    const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
-    RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, tm_h_shared, tm_ws2, g, grid, s));
-  }
-  RMOE_TRY(record(MOE_STAGE_SHARED_EXPERT));
-  if (c.I_shared > 0 && !fused) {
-    {  // hs = silu(x . Ws13g^T) * (x . Ws13u^T)
+  if (use_swap(c)) {
+    RMOE_TRY(swap_gemms(c, x, xp, h, hs, Y, tm_w13, tm_w2, tm_ws13, tm_ws2, offsets, o, a, sms,
+                        record, s));
+  } else {
+    RMOE_TRY(record(MOE_STAGE_EXPERT_UP));
+    {  // h = silu(A . W13g^T) * (A . W13u^T) per group: A = gathered rows (experts), x (shared)
       GemmArgs g = a;
-      g.single_rows = c.T;
-      g.n_tiles = (c.I_shared + 127) / 128;
+      g.mtile_start = mtiles;
+      g.row_start = offsets;
+      g.num_groups = groups;
+      if (fused) {
+        g.alt_group = c.E;
+        g.alt_row0 = (int)R;
+      }
+      g.n_tiles = (c.I + 127) / 128;
       g.k_steps = c.H / 64;
       g.n_out_tile = 128;
-      g.b_second = c.I_shared;
-      g.out = hs;
-      g.ldo = c.I_shared;
-      g.n_valid = c.I_shared;
-      const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
-      RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_x, tm_ws13, tm_x, tm_ws13, g,
-                                   std::min(sms, 2 * tiles), s));
+      g.b_second = c.I;
+      g.out = h;
+      g.ldo = c.I;
+      g.n_valid = c.I;
+      const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
+      RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_xp, tm_w13, tm_x, tm_ws13, g, grid, s));
     }
-    {  // Y[t*slots + top_k] = hs . Ws2^T  (unscaled)
+    RMOE_TRY(record(MOE_STAGE_EXPERT_DOWN));
+    {  // Y[t*slots + j] = w_tj * (h . W2^T) per expert; shared rows to slot top_k, unscaled
       GemmArgs g = a;
-      g.single_rows = c.T;
+      g.mtile_start = mtiles;
+      g.row_start = offsets;
+      g.num_groups = groups;
+      if (fused) {
+        g.alt_group = c.E;
+        g.alt_row0 = (int)R;
+      }
       g.n_tiles = (c.H + 255) / 256;
-      g.k_steps = c.I_shared / 64;
+      g.k_steps = c.I / 64;
       g.n_out_tile = 256;
       g.b_second = 128;
       g.out = Y;
       g.ldo = c.H;
       g.n_valid = c.H;
+      g.row_scale = o.w_of;
+      g.dest_pos = o.pos_of;
       g.dest_mul = slots;
       g.dest_add = c.top_k;
-      const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
-      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_hs, tm_ws2, tm_hs, tm_ws2, g,
-                                   std::min(sms, 2 * tiles), s));
+      const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
+      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, tm_h_shared, tm_ws2, g, grid, s));
+    }
+    RMOE_TRY(record(MOE_STAGE_SHARED_EXPERT));
+    if (c.I_shared > 0 && !fused) {
+      {  // hs = silu(x . Ws13g^T) * (x . Ws13u^T)
+        GemmArgs g = a;
+        g.single_rows = c.T;
+        g.n_tiles = (c.I_shared + 127) / 128;
+        g.k_steps = c.H / 64;
+        g.n_out_tile = 128;
+        g.b_second = c.I_shared;
+        g.out = hs;
+        g.ldo = c.I_shared;
+        g.n_valid = c.I_shared;
+        const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
+        RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_x, tm_ws13, tm_x, tm_ws13, g,
+                                     std::min(sms, 2 * tiles), s));
+      }
+      {  // Y[t*slots + top_k] = hs . Ws2^T  (unscaled)
+        GemmArgs g = a;
+        g.single_rows = c.T;
+        g.n_tiles = (c.H + 255) / 256;
+        g.k_steps = c.I_shared / 64;
+        g.n_out_tile = 256;
+        g.b_second = 128;
+        g.out = Y;
+        g.ldo = c.H;
+        g.n_valid = c.H;
+        g.dest_mul = slots;
+        g.dest_add = c.top_k;
+        const int tiles = (int)((T + MTILE - 1) / MTILE) * g.n_tiles;
+        RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_hs, tm_ws2, tm_hs, tm_ws2, g,
+                                     std::min(sms, 2 * tiles), s));
+      }
     }
   }
   RMOE_TRY(record(MOE_STAGE_COMBINE));

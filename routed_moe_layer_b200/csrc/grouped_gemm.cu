@@ -411,18 +411,23 @@ cudaError_t launch_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUt
 
 }  // namespace
 
-cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K) {
+cudaError_t make_tmap_2d_box(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K,
+                             uint32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   const cuuint64_t dims[2] = {K, rows};
   const cuuint64_t strides[1] = {K * 2};
-  const cuuint32_t box[2] = {BK, BM};
+  const cuuint32_t box[2] = {BK, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K) {
+  return make_tmap_2d_box(map, base, rows, K, BM);
 }
 
 cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, uint64_t groups, uint64_t n_rows,

@@ -95,6 +95,9 @@ struct GemmArgs {
 // A: 2D map over [rows, K] bf16, box 64 x 128, 128B swizzle.
 // B: 3D map over [groups, N_rows, K] bf16, box 64 x 128 x 1, 128B swizzle.
 cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K);
+// The same with a box of box_rows rows (the token operand of the swapped GEMM: 32).
+cudaError_t make_tmap_2d_box(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K,
+                             uint32_t box_rows);
 cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, uint64_t groups, uint64_t n_rows,
                          uint64_t K);
 
@@ -102,6 +105,15 @@ cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, uint64_t groups, ui
 cudaError_t launch_grouped_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
                                 const CUtensorMap& tmA2, const CUtensorMap& tmB2,
                                 const GemmArgs& args, int grid, cudaStream_t stream);
+
+// Swapped operands for few rows per group (grouped_gemm_swap.cu): tmW is the
+// weights' 3D map (box 64 x 128 x 1), tmX the rows' 2D map with 32-row boxes;
+// groups come from args.row_start (null: one group of args.single_rows rows)
+// in chunks of 128 rows; args.n_out_tile must be 128, args.n_tiles counts
+// 128-row weight tiles, args.b_second is the up half's first row (SwiGLU).
+cudaError_t launch_grouped_gemm_swap(int epi, const CUtensorMap& tmW, const CUtensorMap& tmX,
+                                     const CUtensorMap& tmW2, const CUtensorMap& tmX2,
+                                     const GemmArgs& args, int grid, cudaStream_t stream);
 
 int num_sms();
 

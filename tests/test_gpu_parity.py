@@ -121,9 +121,13 @@ def test_permute_reports_bad_expert_id(T):
 
 
 # ------------------------------------------------------------------ forward
+# up to 64 rows per expert on average (T*k <= 64*E) the expert GEMMs run with
+# swapped operands, above it on 256-row tiles: the cases cover both
 FORWARD_CASES = [
     # T, H, E, I, I_shared, k, G, g
     (1, 256, 16, 128, 128, 4, 4, 2),
+    (129, 256, 128, 192, 192, 8, 4, 2),     # swapped: I tail inside a 128-row weight tile
+    (64, 320, 64, 128, 64, 6, 8, 3),        # swapped: H tail, separate shared-expert GEMMs
     (100, 256, 16, 128, 128, 4, 4, 2),
     (300, 512, 32, 192, 64, 8, 4, 2),       # I not a multiple of 128: SwiGLU N tail
     (700, 320, 16, 128, 128, 4, 4, 2),      # H not a multiple of 256: down/combine N tail
@@ -170,10 +174,12 @@ def test_forward_in_place_residual():
     assert torch.equal(buf, ref)
 
 
-def test_forward_hot_experts_many_tiles():
+@pytest.mark.parametrize("T", [1000, 1500])
+def test_forward_hot_experts_many_tiles(T):
     # a bias of +10 on 8 experts (2 groups) sends every token to them: those
-    # experts get T rows (many full tiles + a tail), the other 120 get none
-    T, H = 1500, 512
+    # experts get T rows (many full tiles or 128-row chunks + a tail), the
+    # other 120 get none; T = 1000 runs the swapped GEMMs, 1500 the tiled ones
+    H = 512
     cfg = BlockConfig(T=T, H=H, I=256, I_shared=128)
     d = inputs.make_block_inputs(T, H, seed=21, I=256, I_shared=128, unit_scale=True)
     hot = [0, 5, 9, 31, 64, 70, 80, 95]
@@ -182,6 +188,21 @@ def test_forward_hot_experts_many_tiles():
     assert all(sorted(r) == hot for r in ids.cpu().tolist())
     rep = parity.check_output(out, ids, parity.np_inputs(d), cfg)
     assert rep["rms_rel"] < 1e-2, rep
+
+
+def test_swapped_and_tiled_gemms_agree():
+    """The same tokens through the swapped GEMMs (a small batch) and through
+    the 256-row tiles (inside a large batch) give the same bits: both add the
+    K steps in the same order and apply the same epilogue arithmetic."""
+    T, H = 2048, 1024
+    cfg = BlockConfig(T=T, H=H)
+    d = _dev(inputs.make_block_inputs(T, H, seed=41, unit_scale=True))
+    big, ids_big, _ = _run(d, cfg)  # 128 rows per expert: tiled
+    n = 300                          # 18.75 rows per expert: swapped
+    small, ids_small, _ = _run(dict(d, x=d["x"][:n].contiguous()), cfg.with_tokens(n))
+    assert torch.equal(ids_small, ids_big[:n])
+    diff = (small.float() - big[:n].float()).abs()
+    assert torch.equal(small, big[:n]), f"max diff {diff.max().item()}, {int((diff > 0).sum())} differ"
 
 
 @pytest.mark.parametrize("wid", [0, 1])
