@@ -66,6 +66,10 @@ bool fuse_shared(const moe_cfg_t& c) { return c.I_shared > 0 && c.I_shared == c.
 // that tiles are not padded to 256 rows.  Decided from the shapes only.
 bool use_swap(const moe_cfg_t& c) { return (int64_t)c.T * c.top_k <= 64LL * c.E; }
 
+// Token rows per item of the swapped GEMMs: 32 when the experts average at
+// most 20 rows (so that few of them need a second chunk), else 128.
+int swap_chunk(const moe_cfg_t& c) { return (int64_t)c.T * c.top_k <= 20LL * c.E ? 32 : 128; }
+
 FwdLayout fwd_layout(const moe_cfg_t& c) {
   FwdLayout L;
   const size_t T = c.T, R = T * c.top_k, E = c.E;
@@ -161,7 +165,8 @@ cudaError_t swap_gemms(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp, __n
   const int slots = slots_per_token(c);
   const bool fused = fuse_shared(c);
   const int groups = c.E + (fused ? 1 : 0);
-  const long long chunk_bound = (long long)(R / 128) + groups + 1;
+  const int chunk = swap_chunk(c);
+  const long long chunk_bound = (long long)(R / chunk) + groups + 1;
   CUtensorMap tm_xp, tm_x, tm_h, tm_h_shared, tm_hs;
   cudaError_t e;
   if ((e = make_tmap_2d_box(&tm_xp, xp, R, c.H, 32)) != cudaSuccess) return e;
@@ -193,7 +198,8 @@ cudaError_t swap_gemms(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp, __n
     g.ldo = c.I;
     g.n_valid = c.I;
     const int grid = (int)std::min<long long>(sms, chunk_bound * g.n_tiles);
-    if ((e = launch_grouped_gemm_swap(EPI_SWIGLU, tm_w13, tm_xp, tm_ws13, tm_x, g, grid, s)) !=
+    if ((e = launch_grouped_gemm_swap(EPI_SWIGLU, chunk, tm_w13, tm_xp, tm_ws13, tm_x, g, grid,
+                                      s)) !=
         cudaSuccess)
       return e;
   }
@@ -218,13 +224,13 @@ cudaError_t swap_gemms(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp, __n
     g.dest_mul = slots;
     g.dest_add = c.top_k;
     const int grid = (int)std::min<long long>(sms, chunk_bound * g.n_tiles);
-    if ((e = launch_grouped_gemm_swap(EPI_ROWSCALE, tm_w2, tm_h, tm_ws2, tm_h_shared, g, grid,
+    if ((e = launch_grouped_gemm_swap(EPI_ROWSCALE, chunk, tm_w2, tm_h, tm_ws2, tm_h_shared, g, grid,
                                       s)) != cudaSuccess)
       return e;
   }
   if ((e = record(MOE_STAGE_SHARED_EXPERT)) != cudaSuccess) return e;
   if (c.I_shared > 0 && !fused) {
-    const long long chunks = (long long)(T + 127) / 128;
+    const long long chunks = (long long)(T + chunk - 1) / chunk;
     {  // hs = silu(x . Ws13g^T) * (x . Ws13u^T)
       GemmArgs g = a;
       g.single_rows = c.T;
@@ -236,7 +242,8 @@ cudaError_t swap_gemms(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp, __n
       g.ldo = c.I_shared;
       g.n_valid = c.I_shared;
       const int grid = (int)std::min<long long>(sms, chunks * g.n_tiles);
-      if ((e = launch_grouped_gemm_swap(EPI_SWIGLU, tm_ws13, tm_x, tm_ws13, tm_x, g, grid, s)) !=
+      if ((e = launch_grouped_gemm_swap(EPI_SWIGLU, chunk, tm_ws13, tm_x, tm_ws13, tm_x, g, grid,
+                                        s)) !=
           cudaSuccess)
         return e;
     }
@@ -252,7 +259,8 @@ cudaError_t swap_gemms(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp, __n
       g.dest_mul = slots;
       g.dest_add = c.top_k;
       const int grid = (int)std::min<long long>(sms, chunks * g.n_tiles);
-      if ((e = launch_grouped_gemm_swap(EPI_ROWSCALE, tm_ws2, tm_hs, tm_ws2, tm_hs, g, grid, s)) !=
+      if ((e = launch_grouped_gemm_swap(EPI_ROWSCALE, chunk, tm_ws2, tm_hs, tm_ws2, tm_hs, g,
+                                        grid, s)) !=
           cudaSuccess)
         return e;
     }

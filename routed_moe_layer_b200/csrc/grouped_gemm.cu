@@ -120,7 +120,9 @@ __device__ __forceinline__ TileCoord cta_part(TileCoord c, uint32_t rank) {
   return c;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
+// silu(g) = g / (1 + e^-g); the same expression as in grouped_gemm_swap.cu, so
+// that both kernels give the same bits.
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // Per-row inputs of the epilogue, read before the accumulator is waited for
 // so that their latency hides behind the MMAs.

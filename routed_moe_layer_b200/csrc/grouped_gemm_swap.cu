@@ -10,7 +10,7 @@
 // expert a 256-row tile would spend 94% of its tensor work on padding and
 // leave the kernel bound by the MMAs instead of by streaming the weights.
 //
-// Work item = (chunk of at most 128 rows of one group, 128 weight rows):
+// Work item = (chunk of at most CHUNK rows of one group, 128 weight rows):
 //   EPI_SWIGLU    weight rows i0.. of the gate half and I+i0.. of the up half
 //                 go to two accumulators (TMEM columns +0 and +128), so that
 //                 the thread holding TMEM lane l has gate and up of output
@@ -18,7 +18,9 @@
 //                 out[r, i0+l] = bf16( silu(gate) * up )
 //   EPI_ROWSCALE  weight rows h0..h0+127 of W2: out[pos[r], h0+l] =
 //                 bf16( row_scale[r] * D[l, r] )
-// Token rows come in 32-row TMA boxes (only the chunk's rows are loaded);
+// CHUNK is 128, or 32 when the experts hold very few rows (more of shared
+// memory then goes to staging the weight stream: 6 or 10 stages instead of 4
+// or 6).  Token rows come in 32-row TMA boxes (only the chunk's rows are loaded);
 // weights in 128-row boxes.  Warp roles: warp 0 one thread issues the TMA
 // loads; warp 1 allocates 512 TMEM columns (two accumulator buffers) and one
 // thread issues the MMAs; warps 2..5 run the epilogue of item i while the MMAs
@@ -30,7 +32,6 @@ namespace rmoe {
 
 namespace {
 
-constexpr int CHUNK = 128;  // token rows per item (the MMA's N, padded to 16)
 constexpr int WM = 128;     // weight rows per item (the MMA's M)
 constexpr int BK = 64;
 constexpr int XBOX = 32;    // token rows per TMA box
@@ -40,18 +41,23 @@ constexpr int MAX_GROUPS = 129;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COLS = 256;            // per accumulator buffer
 constexpr int W_BYTES = WM * BK * 2;          // one weight tile
-constexpr int X_BYTES = CHUNK * BK * 2;       // token tile (up to 128 rows)
 constexpr int XBOX_BYTES = XBOX * BK * 2;
-constexpr int MAX_STAGES = 6;
+constexpr int MAX_STAGES = 10;
 constexpr unsigned FULL = 0xffffffffu;
 
-template <int EPI>
+// CHUNK = token rows per item (the MMA's N, padded to 16): 128, or 32 when the
+// experts hold very few rows, which frees shared memory for deeper staging of
+// the weight stream.
+template <int EPI, int CHUNK>
 struct Shape {
   static constexpr int NW = EPI == EPI_SWIGLU ? 2 : 1;  // weight tiles per stage
+  static constexpr int X_BYTES = CHUNK * BK * 2;        // token tile
   static constexpr int STAGE_BYTES = NW * W_BYTES + X_BYTES;
-  static constexpr int STAGES = EPI == EPI_SWIGLU ? 4 : 6;
+  static constexpr int STAGES = EPI == EPI_SWIGLU ? (CHUNK == 32 ? 6 : 4) : (CHUNK == 32 ? 10 : 6);
+  static_assert(STAGES <= MAX_STAGES, "stage count");
 };
 
+template <int CHUNK>
 struct __align__(8) Tail {
   uint64_t full[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
@@ -66,9 +72,10 @@ struct __align__(8) Tail {
   int tok_d[EPI_WARPS][CHUNK];    //   chunk's row weights and output rows
 };
 
-template <int EPI>
+template <int EPI, int CHUNK>
 constexpr size_t smem_bytes() {
-  return 1024 + (size_t)Shape<EPI>::STAGES * Shape<EPI>::STAGE_BYTES + sizeof(Tail);
+  return 1024 + (size_t)Shape<EPI, CHUNK>::STAGES * Shape<EPI, CHUNK>::STAGE_BYTES +
+         sizeof(Tail<CHUNK>);
 }
 
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity,
@@ -84,6 +91,7 @@ struct Item {
   int g, row0, rows, mt;
 };
 
+template <int CHUNK>
 __device__ __forceinline__ Item item_coord(int item, int n_tiles, int groups, const int* cs,
                                            const int* rs) {
   Item it;
@@ -103,21 +111,23 @@ __device__ __forceinline__ Item item_coord(int item, int n_tiles, int groups, co
   return it;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
+// silu(g) = g / (1 + e^-g); the same expression as in grouped_gemm.cu, so that
+// both kernels give the same bits.
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-template <int EPI>
+template <int EPI, int CHUNK>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmW,
                              const __grid_constant__ CUtensorMap tmX,
                              const __grid_constant__ CUtensorMap tmW2,
                              const __grid_constant__ CUtensorMap tmX2, const GemmArgs args) {
-  using S = Shape<EPI>;
+  using S = Shape<EPI, CHUNK>;
   pdl_launch_dependents();
   pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  Tail& st = *reinterpret_cast<Tail*>(smem + (size_t)S::STAGES * S::STAGE_BYTES);
+  Tail<CHUNK>& st = *reinterpret_cast<Tail<CHUNK>*>(smem + (size_t)S::STAGES * S::STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // group table: expert row offsets, or one group of single_rows rows
@@ -196,7 +206,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t armed = 0, armed_parity = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < total; item += gridDim.x) {
-        const Item it = item_coord(item, args.n_tiles, groups, st.ch_start, st.row_start);
+        const Item it = item_coord<CHUNK>(item, args.n_tiles, groups, st.ch_start, st.row_start);
         const bool alt = it.g == args.alt_group;
         const CUtensorMap* mw = alt ? &tmW2 : &tmW;
         const CUtensorMap* mx = alt ? &tmX2 : &tmX;
@@ -241,7 +251,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < total; item += gridDim.x) {
-        const Item it = item_coord(item, args.n_tiles, groups, st.ch_start, st.row_start);
+        const Item it = item_coord<CHUNK>(item, args.n_tiles, groups, st.ch_start, st.row_start);
         const int n_pad = (it.rows + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(WM, n_pad);
         if (!mbar_wait(&st.tempty[acc], acc_phase ^ 1u, wc, 41)) break;
@@ -287,7 +297,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
-      const Item it = item_coord(item, args.n_tiles, groups, st.ch_start, st.row_start);
+      const Item it = item_coord<CHUNK>(item, args.n_tiles, groups, st.ch_start, st.row_start);
       const bool alt = it.g == args.alt_group;
       const int n_pad = (it.rows + 15) & ~15;
       const int col = it.mt * args.n_out_tile + l;  // output column of this thread
@@ -366,34 +376,37 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int EPI>
+template <int EPI, int CHUNK>
 cudaError_t launch_swap(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtensorMap& tmW2,
                         const CUtensorMap& tmX2, const GemmArgs& args, int grid,
                         cudaStream_t stream) {
-  static cudaError_t attr =
-      cudaFuncSetAttribute(grouped_gemm_swap_kernel<EPI>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes<EPI>());
+  constexpr size_t smem = smem_bytes<EPI, CHUNK>();
+  static_assert(smem <= 227 * 1024, "shared memory");
+  static cudaError_t attr = cudaFuncSetAttribute(
+      grouped_gemm_swap_kernel<EPI, CHUNK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (attr != cudaSuccess) return attr;
   if (grid < 1) grid = 1;
-  return launch_chained(grouped_gemm_swap_kernel<EPI>, dim3(grid), dim3(THREADS),
-                        smem_bytes<EPI>(), stream, tmW, tmX, tmW2, tmX2, args);
+  return launch_chained(grouped_gemm_swap_kernel<EPI, CHUNK>, dim3(grid), dim3(THREADS), smem,
+                        stream, tmW, tmX, tmW2, tmX2, args);
 }
 
 }  // namespace
 
-cudaError_t launch_grouped_gemm_swap(int epi, const CUtensorMap& tmW, const CUtensorMap& tmX,
-                                     const CUtensorMap& tmW2, const CUtensorMap& tmX2,
-                                     const GemmArgs& args, int grid, cudaStream_t stream) {
+cudaError_t launch_grouped_gemm_swap(int epi, int chunk, const CUtensorMap& tmW,
+                                     const CUtensorMap& tmX, const CUtensorMap& tmW2,
+                                     const CUtensorMap& tmX2, const GemmArgs& args, int grid,
+                                     cudaStream_t stream) {
   if (args.row_start && args.num_groups > MAX_GROUPS) return cudaErrorInvalidValue;
   if (args.n_out_tile != WM) return cudaErrorInvalidValue;
-  switch (epi) {
-    case EPI_SWIGLU:
-      return launch_swap<EPI_SWIGLU>(tmW, tmX, tmW2, tmX2, args, grid, stream);
-    case EPI_ROWSCALE:
-      return launch_swap<EPI_ROWSCALE>(tmW, tmX, tmW2, tmX2, args, grid, stream);
-    default:
-      return cudaErrorInvalidValue;
-  }
+  if (epi == EPI_SWIGLU && chunk == 32)
+    return launch_swap<EPI_SWIGLU, 32>(tmW, tmX, tmW2, tmX2, args, grid, stream);
+  if (epi == EPI_SWIGLU && chunk == 128)
+    return launch_swap<EPI_SWIGLU, 128>(tmW, tmX, tmW2, tmX2, args, grid, stream);
+  if (epi == EPI_ROWSCALE && chunk == 32)
+    return launch_swap<EPI_ROWSCALE, 32>(tmW, tmX, tmW2, tmX2, args, grid, stream);
+  if (epi == EPI_ROWSCALE && chunk == 128)
+    return launch_swap<EPI_ROWSCALE, 128>(tmW, tmX, tmW2, tmX2, args, grid, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace rmoe

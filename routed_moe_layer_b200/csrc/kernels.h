@@ -109,11 +109,13 @@ cudaError_t launch_grouped_gemm(int epi, const CUtensorMap& tmA, const CUtensorM
 // Swapped operands for few rows per group (grouped_gemm_swap.cu): tmW is the
 // weights' 3D map (box 64 x 128 x 1), tmX the rows' 2D map with 32-row boxes;
 // groups come from args.row_start (null: one group of args.single_rows rows)
-// in chunks of 128 rows; args.n_out_tile must be 128, args.n_tiles counts
-// 128-row weight tiles, args.b_second is the up half's first row (SwiGLU).
-cudaError_t launch_grouped_gemm_swap(int epi, const CUtensorMap& tmW, const CUtensorMap& tmX,
-                                     const CUtensorMap& tmW2, const CUtensorMap& tmX2,
-                                     const GemmArgs& args, int grid, cudaStream_t stream);
+// in chunks of `chunk` (32 or 128) rows; args.n_out_tile must be 128,
+// args.n_tiles counts 128-row weight tiles, args.b_second is the up half's
+// first row (SwiGLU).
+cudaError_t launch_grouped_gemm_swap(int epi, int chunk, const CUtensorMap& tmW,
+                                     const CUtensorMap& tmX, const CUtensorMap& tmW2,
+                                     const CUtensorMap& tmX2, const GemmArgs& args, int grid,
+                                     cudaStream_t stream);
 
 int num_sms();
 

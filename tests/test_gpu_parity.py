@@ -122,7 +122,8 @@ def test_permute_reports_bad_expert_id(T):
 
 # ------------------------------------------------------------------ forward
 # up to 64 rows per expert on average (T*k <= 64*E) the expert GEMMs run with
-# swapped operands, above it on 256-row tiles: the cases cover both
+# swapped operands (32-row chunks up to 20 rows per expert, else 128-row
+# chunks), above it on 256-row tiles: the cases cover all three
 FORWARD_CASES = [
     # T, H, E, I, I_shared, k, G, g
     (1, 256, 16, 128, 128, 4, 4, 2),
@@ -174,11 +175,12 @@ def test_forward_in_place_residual():
     assert torch.equal(buf, ref)
 
 
-@pytest.mark.parametrize("T", [1000, 1500])
+@pytest.mark.parametrize("T", [300, 1000, 1500])
 def test_forward_hot_experts_many_tiles(T):
     # a bias of +10 on 8 experts (2 groups) sends every token to them: those
-    # experts get T rows (many full tiles or 128-row chunks + a tail), the
-    # other 120 get none; T = 1000 runs the swapped GEMMs, 1500 the tiled ones
+    # experts get T rows (many full tiles or chunks + a tail), the other 120
+    # get none; T = 300 runs the swapped GEMMs with 32-row chunks, 1000 with
+    # 128-row chunks, 1500 the tiled GEMMs
     H = 512
     cfg = BlockConfig(T=T, H=H, I=256, I_shared=128)
     d = inputs.make_block_inputs(T, H, seed=21, I=256, I_shared=128, unit_scale=True)
