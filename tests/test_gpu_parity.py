@@ -66,6 +66,24 @@ def test_router_on_workloads(wid):
     np.testing.assert_allclose(w.sum(1).cpu().numpy(), 2.5, rtol=1e-5)
 
 
+@pytest.mark.parametrize("H,E,k,G,g", [(1024, 128, 8, 4, 2), (512, 64, 6, 8, 3),
+                                       (256, 96, 16, 4, 4), (256, 32, 4, 1, 1)])
+def test_router_batch_isolation(H, E, k, G, g):
+    """A token's routing does not depend on the other tokens of the call: the
+    first tokens of a large batch, routed alone, give the same bits (and the
+    large batch matches the oracle)."""
+    T, n = 4133, 777
+    cfg = BlockConfig(T=T, H=H, E=E, top_k=k, n_group=G, topk_group=g)
+    d = inputs.make_block_inputs(T, H, seed=E + k, E=E, I=64, I_shared=0, unit_scale=True)
+    dd = _dev(d)
+    ids, w = ops.route(dd["x"], dd["Wr"], dd["bias"], cfg)
+    ids_s, w_s = ops.route(dd["x"][:n].contiguous(), dd["Wr"], dd["bias"], cfg.with_tokens(n))
+    torch.cuda.synchronize()
+    assert torch.equal(ids_s, ids[:n]) and torch.equal(w_s, w[:n])
+    rep = parity.check_routing(ids, w, *[parity.to_np(d[m]) for m in ("x", "Wr", "bias")], cfg)
+    assert rep["near_ties"] <= max(2, T // 20)
+
+
 def test_router_bias_forces_selection_not_weights():
     T, H = 200, 512
     cfg = BlockConfig(T=T, H=H)
