@@ -42,7 +42,9 @@ notes of the repository):
   * experts outside the kept groups are excluded (score -inf), not zeroed;
   * group scores use the bias-corrected scores c, like the expert choice;
   * ``norm_topk_prob`` is on; the denominator has no epsilon guard;
-  * ids are returned in selection order (descending c).
+  * ids are returned in selection order (descending c);
+  * the padding mask is per token: a padding token takes no routed expert
+    (id -1, weight 0) and keeps the shared expert (see ``apply_token_mask``).
 """
 
 from __future__ import annotations
@@ -161,11 +163,35 @@ def routing_weights(s: np.ndarray, ids: np.ndarray, routed_scaling_factor: float
     return routed_scaling_factor * sel
 
 
-def route(x, Wr, bias, cfg: MoeConfig):
+def apply_token_mask(ids: np.ndarray, w: np.ndarray, margin: np.ndarray, token_mask):
+    """Padding mask ([S2] "MoE 实现的源码级要点": in the forward the padding mask
+    acts on the routing scores, which are then renormalised).
+
+    Reading: the mask is per token (nonzero = real token, 0 = padding).  A
+    padding token's routing scores are masked to zero, so it takes no routed
+    expert: id -1 and weight 0 (renormalising an all-zero row keeps it zero).
+    A real token's choice and weights are unchanged (its own scores are not
+    masked, and renormalising them again is the identity).  The shared expert
+    is dense and still applies to every token.
+    Returns new (ids, w, margin); a padding token's margin is +inf (no choice).
+    """
+    real = np.asarray(token_mask).reshape(-1) != 0
+    ids = np.array(ids, dtype=np.int32, copy=True)
+    w = np.array(w, dtype=np.float64, copy=True)
+    margin = np.array(margin, dtype=np.float64, copy=True)
+    ids[~real] = -1
+    w[~real] = 0.0
+    margin[~real] = np.inf
+    return ids, w, margin
+
+
+def route(x, Wr, bias, cfg: MoeConfig, token_mask=None):
     """Full router: returns (ids int32 [T,k], w float64 [T,k], margin [T], s fp32 [T,E])."""
     _, s, c = router_scores(x, Wr, bias)
     ids, margin = group_limited_topk(c, cfg.n_group, cfg.topk_group, cfg.top_k)
     w = routing_weights(s, ids, cfg.routed_scaling_factor, cfg.norm_topk_prob)
+    if token_mask is not None:
+        ids, w, margin = apply_token_mask(ids, w, margin, token_mask)
     return ids, w, margin, s
 
 
@@ -213,7 +239,7 @@ def swiglu_mlp(x: np.ndarray, w13: np.ndarray, w2: np.ndarray) -> np.ndarray:
 
 
 def moe_forward(x, Wr, bias, w13, w2, ws13, ws2, cfg: MoeConfig,
-                residual=None, ids=None):
+                residual=None, ids=None, token_mask=None):
     """Block output in float64 [T,H].
 
     out = sum_i w_i * Expert_{ids_i}(x)          (fp32 scatter-weighted restore, [S2])
@@ -222,7 +248,8 @@ def moe_forward(x, Wr, bias, w13, w2, ws13, ws2, cfg: MoeConfig,
 
     ``ids`` may be given (e.g. to evaluate near-tie tokens under another
     implementation's choice); the weights are then recomputed from this
-    oracle's own raw scores for those ids.
+    oracle's own raw scores for those ids.  ``token_mask`` (per token,
+    0 = padding) removes the routed part of padding tokens (``apply_token_mask``).
     Returns (out, ids, w, margin).
     """
     _, s, c = router_scores(x, Wr, bias)
@@ -231,7 +258,11 @@ def moe_forward(x, Wr, bias, w13, w2, ws13, ws2, cfg: MoeConfig,
     else:
         ids = np.asarray(ids, dtype=np.int32)
         _, margin = group_limited_topk(c, cfg.n_group, cfg.topk_group, cfg.top_k)
+    if token_mask is not None:
+        ids = np.where((np.asarray(token_mask).reshape(-1) != 0)[:, None], ids, 0)
     w = routing_weights(s, ids, cfg.routed_scaling_factor, cfg.norm_topk_prob)
+    if token_mask is not None:
+        ids, w, margin = apply_token_mask(ids, w, margin, token_mask)
     T, H = x.shape
     out = np.zeros((T, H), dtype=np.float64)
     for e in range(w13.shape[0]):
@@ -248,15 +279,16 @@ def moe_forward(x, Wr, bias, w13, w2, ws13, ws2, cfg: MoeConfig,
 
 
 def moe_forward_tokens(tokens, x, Wr, bias, w13, w2, ws13, ws2, cfg: MoeConfig,
-                       residual=None, ids=None):
+                       residual=None, ids=None, token_mask=None):
     """``moe_forward`` restricted to the token indices ``tokens`` (each token
     is computed in isolation, so this equals the corresponding rows of the
     full output).  Used to check full-size runs on a sample of outputs."""
     tokens = np.asarray(tokens, dtype=np.int64)
     res = None if residual is None else residual[tokens]
     sub_ids = None if ids is None else np.asarray(ids)[tokens]
+    sub_mask = None if token_mask is None else np.asarray(token_mask).reshape(-1)[tokens]
     return moe_forward(x[tokens], Wr, bias, w13, w2, ws13, ws2, cfg,
-                       residual=res, ids=sub_ids)
+                       residual=res, ids=sub_ids, token_mask=sub_mask)
 
 
 # ----------------------------------------------------------------------------

@@ -61,6 +61,22 @@ def _scaled_shared(*args, **kw):
 
 
 _ORIG_FWD = om.moe_forward
+_ORIG_MASK = om.apply_token_mask
+
+
+def _mask_ignored(ids, w, margin, token_mask):
+    return ids, w, margin
+
+
+def _forward_mask_kills_shared(*args, **kw):
+    out, ids, w, m = _ORIG_FWD(*args, **kw)
+    mask = kw.get("token_mask")
+    if mask is not None:
+        res = kw.get("residual")
+        pad = np.asarray(mask).reshape(-1) == 0
+        out = out.copy()
+        out[pad] = 0.0 if res is None else np.asarray(res, dtype=np.float64)[pad]
+    return out, ids, w, m
 
 PIN_TESTS = [
     lambda: pins.test_hand_worked_golden_example(),
@@ -71,6 +87,7 @@ PIN_TESTS = [
     lambda: pins.test_identical_experts_give_scaled_dense_mlp(),
     lambda: pins.test_single_expert_is_textbook_swiglu_plus_shared(),
     lambda: pins.test_swiglu_gate_up_order_and_w2_orientation(),
+    lambda: pins.test_padding_mask_keeps_only_the_shared_expert(),
 ]
 
 MUTATIONS = {
@@ -87,6 +104,8 @@ MUTATIONS = {
     "w2_misoriented": [(om, "swiglu_mlp", _w2_transposed_use),
                        (pins, "swiglu_mlp", _w2_transposed_use)],
     "shared_expert_scaled": [(pins, "moe_forward", _scaled_shared)],
+    "padding_mask_ignored": [(om, "apply_token_mask", _mask_ignored)],
+    "padding_drops_shared_expert": [(pins, "moe_forward", _forward_mask_kills_shared)],
 }
 
 

@@ -289,6 +289,44 @@ def test_residual_and_given_ids():
     np.testing.assert_allclose(w_g, w[:, ::-1], rtol=1e-15)
 
 
+def test_padding_mask_keeps_only_the_shared_expert():
+    # [S2] "MoE 实现的源码级要点": the padding mask acts on the routing scores, which
+    # are renormalised.  A padding token takes no routed expert (id -1, weight 0)
+    # and keeps the dense shared expert; real tokens are untouched.
+    x, Wr, bias, w13, w2, ws13, ws2, cfg = _block(T=48)
+    mask = np.ones(48, dtype=np.uint8)
+    mask[[0, 7, 8, 30, 47]] = 0
+    res = np.full_like(x, 0.25)
+    full, ids0, w0, m0 = moe_forward(x, Wr, bias, w13, w2, ws13, ws2, cfg, residual=res)
+    out, ids, w, margin = moe_forward(x, Wr, bias, w13, w2, ws13, ws2, cfg, residual=res,
+                                      token_mask=mask)
+    pad = mask == 0
+    # padding tokens: a textbook SwiGLU MLP of the shared weights, plus the residual
+    F = torch.nn.functional
+    xt = torch.from_numpy(x[pad]).double()
+    Is = cfg.I_shared
+    g = torch.from_numpy(ws13[:Is]).double()
+    u = torch.from_numpy(ws13[Is:]).double()
+    sh = F.linear(F.silu(F.linear(xt, g)) * F.linear(xt, u), torch.from_numpy(ws2).double())
+    np.testing.assert_allclose(out[pad], sh.numpy() + 0.25, rtol=1e-12, atol=1e-12)
+    assert np.all(ids[pad] == -1) and np.all(w[pad] == 0) and np.all(np.isinf(margin[pad]))
+    # real tokens: bit for bit what the unmasked block gives
+    assert np.array_equal(out[~pad], full[~pad])
+    assert np.array_equal(ids[~pad], ids0[~pad]) and np.array_equal(w[~pad], w0[~pad])
+    # all padding: only the shared expert anywhere; no padding: the unmasked block
+    out_all, ids_all, _, _ = moe_forward(x, Wr, bias, w13, w2, ws13, ws2, cfg,
+                                         token_mask=np.zeros(48, dtype=np.uint8))
+    assert np.all(ids_all == -1)
+    np.testing.assert_allclose(out_all, swiglu_mlp(x, ws13, ws2), rtol=1e-14)
+    out_none, _, _, _ = moe_forward(x, Wr, bias, w13, w2, ws13, ws2, cfg, residual=res,
+                                    token_mask=np.ones(48, dtype=np.uint8))
+    assert np.array_equal(out_none, full)
+    # the sampled form gives the same rows
+    sub, _, _, _ = moe_forward_tokens([7, 9, 30], x, Wr, bias, w13, w2, ws13, ws2, cfg,
+                                      residual=res, token_mask=mask)
+    np.testing.assert_allclose(sub, out[[7, 9, 30]], rtol=1e-13, atol=1e-14)
+
+
 def test_rmsnorm_unit_rms_and_bf16_rounding():
     rng = np.random.default_rng(2)
     x = rng.standard_normal((10, 256)) * 3.0
