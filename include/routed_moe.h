@@ -98,6 +98,10 @@ typedef struct {
                              the last stage.  Each recorded event orders the kernels around it
                              strictly, so record only the boundaries you time. */
   int64_t wait_timeout_ns;/* limit of every device-side wait; 0 = 2 s */
+  const uint8_t* token_mask; /* device uint8 [T] or NULL (all real): padding mask ([S2] "MoE
+                             实现的源码级要点": the mask acts on the routing scores, which are
+                             renormalised); a token with mask 0 takes no routed expert (id -1,
+                             weight 0) and its output is the shared expert (+ residual) */
 } moe_forward_opts_t;
 
 /* Human-readable name of a status code; never NULL. */
@@ -126,6 +130,19 @@ MOE_API size_t moe_workspace_bytes(const moe_cfg_t* cfg);
 MOE_API int32_t moe_route(const void* x, const float* Wr, const float* bias, const moe_cfg_t* cfg,
                   int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes,
                   void* stream);
+
+/* moe_route with a per-token padding mask ([S2] "MoE 实现的源码级要点": the
+ * padding mask acts on the routing scores, which are renormalised):
+ *   token_mask device uint8 [T]: 0 = padding.  A padding token's routing
+ *              scores are masked to zero, so it takes no expert: its ids are
+ *              -1 and its weights 0 (an all-zero row stays zero when
+ *              renormalised).  Real tokens are routed exactly as by moe_route.
+ * Other arguments, workspace and errors as moe_route; token_mask NULL is
+ * moe_route. */
+MOE_API int32_t moe_route_masked(const void* x, const float* Wr, const float* bias,
+                                 const uint8_t* token_mask, const moe_cfg_t* cfg,
+                                 int32_t* topk_ids, float* topk_w, void* workspace,
+                                 size_t workspace_bytes, void* stream);
 
 /* Token -> expert permutation ([S2] "_reorder_tokens": tokens regrouped per
  * expert before the grouped GEMMs).  Rows are ordered by expert, then by

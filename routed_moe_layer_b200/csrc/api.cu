@@ -167,18 +167,19 @@ cudaError_t swap_gemms(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp, __n
   const int groups = c.E + (fused ? 1 : 0);
   const int chunk = swap_chunk(c);
   const long long chunk_bound = (long long)(R / chunk) + groups + 1;
-  CUtensorMap tm_xp, tm_x, tm_h, tm_h_shared, tm_hs;
+  // h holds the routed rows, then (fused) the shared group's T rows; the
+  // shared group starts at expert_offsets[E], which is below T*top_k when
+  // rows are dropped (padding tokens, rejected ids), so the down projection
+  // reads the shared rows where they are, through the map of all of h
+  const size_t h_rows = R + (fused ? T : 0);
+  CUtensorMap tm_xp, tm_x, tm_h, tm_hs;
   cudaError_t e;
   if ((e = make_tmap_2d_box(&tm_xp, xp, R, c.H, 32)) != cudaSuccess) return e;
-  if ((e = make_tmap_2d_box(&tm_h, h, R, c.I, 32)) != cudaSuccess) return e;
-  tm_x = tm_h_shared = tm_hs = tm_xp;  // unused unless there is a shared expert
+  if ((e = make_tmap_2d_box(&tm_h, h, h_rows, c.I, 32)) != cudaSuccess) return e;
+  tm_x = tm_hs = tm_xp;  // unused unless there is a shared expert
   if (c.I_shared > 0) {
     if ((e = make_tmap_2d_box(&tm_x, x, T, c.H, 32)) != cudaSuccess) return e;
-    if (fused) {
-      if ((e = make_tmap_2d_box(&tm_h_shared, h + R * c.I, T, c.I, 32)) != cudaSuccess) return e;
-    } else {
-      if ((e = make_tmap_2d_box(&tm_hs, hs, T, c.I_shared, 32)) != cudaSuccess) return e;
-    }
+    if (!fused && (e = make_tmap_2d_box(&tm_hs, hs, T, c.I_shared, 32)) != cudaSuccess) return e;
   }
   if ((e = record(MOE_STAGE_EXPERT_UP)) != cudaSuccess) return e;
   {  // h[r, i] = silu(W13g[i] . x_r) * (W13u[i] . x_r) per group (shared expert: group E)
@@ -186,9 +187,9 @@ cudaError_t swap_gemms(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp, __n
     g.mtile_start = o.mtile_start;
     g.row_start = offsets;
     g.num_groups = groups;
-    if (fused) {
+    if (fused) {  // shared rows: A from x at (row - group start)
       g.alt_group = c.E;
-      g.alt_row0 = (int)R;
+      g.alt_rebase = 1;
     }
     g.n_tiles = (c.I + 127) / 128;
     g.k_steps = c.H / 64;
@@ -209,9 +210,9 @@ cudaError_t swap_gemms(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp, __n
     g.mtile_start = o.mtile_start;
     g.row_start = offsets;
     g.num_groups = groups;
-    if (fused) {
+    if (fused) {  // shared rows: A from h at their own rows, weights ws2, unscaled
       g.alt_group = c.E;
-      g.alt_row0 = (int)R;
+      g.alt_rebase = 0;
     }
     g.n_tiles = (c.H + 127) / 128;
     g.k_steps = c.I / 64;
@@ -224,7 +225,7 @@ cudaError_t swap_gemms(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp, __n
     g.dest_mul = slots;
     g.dest_add = c.top_k;
     const int grid = (int)std::min<long long>(sms, chunk_bound * g.n_tiles);
-    if ((e = launch_grouped_gemm_swap(EPI_ROWSCALE, chunk, tm_w2, tm_h, tm_ws2, tm_h_shared, g, grid,
+    if ((e = launch_grouped_gemm_swap(EPI_ROWSCALE, chunk, tm_w2, tm_h, tm_ws2, tm_h, g, grid,
                                       s)) != cudaSuccess)
       return e;
   }
@@ -295,12 +296,13 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
   const int slots = slots_per_token(c);
   const bool fused = fuse_shared(c);
   const size_t h_rows = R + (fused ? T : 0);
-  CUtensorMap tm_xp, tm_w13, tm_h, tm_h_shared, tm_w2, tm_x, tm_ws13, tm_hs, tm_ws2;
+  CUtensorMap tm_xp, tm_w13, tm_h, tm_w2, tm_x, tm_ws13, tm_hs, tm_ws2;
   RMOE_TRY(make_tmap_2d(&tm_xp, xp, R, c.H));
   RMOE_TRY(make_tmap_3d(&tm_w13, w13, c.E, 2 * (uint64_t)c.I, c.H));
-  RMOE_TRY(make_tmap_2d(&tm_h, h, R, c.I));
-  // the shared group's rows of h (rows R..R+T-1), re-based to row 0
-  if (fused) RMOE_TRY(make_tmap_2d(&tm_h_shared, h + R * c.I, T, c.I));
+  // all of h: the routed rows, then (fused) the shared group's T rows, which
+  // start at expert_offsets[E] -- below T*top_k when rows are dropped (padding
+  // tokens, rejected ids) -- and are read where they are
+  RMOE_TRY(make_tmap_2d(&tm_h, h, h_rows, c.I));
   RMOE_TRY(make_tmap_3d(&tm_w2, w2, c.E, c.H, c.I));
   if (c.I_shared > 0) {
     RMOE_TRY(make_tmap_2d(&tm_x, x, T, c.H));
@@ -310,7 +312,6 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
   } else {
     tm_x = tm_ws13 = tm_ws2 = tm_xp;  // unused second maps
   }
-  if (!fused) tm_h_shared = tm_h;  // unused
   const int sms = num_sms();
 
   auto record = [&](int i) -> cudaError_t {
@@ -320,6 +321,7 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
   RMOE_TRY(record(MOE_STAGE_ROUTER));
   RouterParams rp = router_params(c);
   rp.clear_status = clear_status ? 1 : 0;
+  rp.mask = opts ? opts->token_mask : nullptr;
   RMOE_TRY(launch_router(x, Wr, bias, rp, ids, tw, at<void>(workspace, L.router), status, timeout,
                          s));
 
@@ -336,6 +338,7 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
   o.slot_stride = slots;
   o.extra_rows = fused ? c.T : 0;
   o.xp = xp;
+  o.mask = rp.mask;
   RMOE_TRY(launch_permute(ids, tw, x, c.T, c.H, c.E, c.top_k, o, s));
 
   // tiles of MTILE rows, each computed by a pair of CTAs; every group adds at
@@ -358,9 +361,9 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
       g.mtile_start = mtiles;
       g.row_start = offsets;
       g.num_groups = groups;
-      if (fused) {
+      if (fused) {  // shared rows: A from x at (row - group start)
         g.alt_group = c.E;
-        g.alt_row0 = (int)R;
+        g.alt_rebase = 1;
       }
       g.n_tiles = (c.I + 127) / 128;
       g.k_steps = c.H / 64;
@@ -378,9 +381,9 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
       g.mtile_start = mtiles;
       g.row_start = offsets;
       g.num_groups = groups;
-      if (fused) {
+      if (fused) {  // shared rows: A from h at their own rows, weights ws2, unscaled
         g.alt_group = c.E;
-        g.alt_row0 = (int)R;
+        g.alt_rebase = 0;
       }
       g.n_tiles = (c.H + 255) / 256;
       g.k_steps = c.I / 64;
@@ -394,7 +397,7 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
       g.dest_mul = slots;
       g.dest_add = c.top_k;
       const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
-      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, tm_h_shared, tm_ws2, g, grid, s));
+      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, tm_h, tm_ws2, g, grid, s));
     }
     RMOE_TRY(record(MOE_STAGE_SHARED_EXPERT));
     if (c.I_shared > 0 && !fused) {
@@ -472,9 +475,9 @@ size_t moe_workspace_bytes(const moe_cfg_t* cfg) {
   return fwd_layout(*cfg).total;
 }
 
-int32_t moe_route(const void* x, const float* Wr, const float* bias, const moe_cfg_t* cfg,
-                  int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes,
-                  void* stream) {
+int32_t moe_route_masked(const void* x, const float* Wr, const float* bias,
+                         const uint8_t* token_mask, const moe_cfg_t* cfg, int32_t* topk_ids,
+                         float* topk_w, void* workspace, size_t workspace_bytes, void* stream) {
   const int32_t st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
@@ -482,9 +485,18 @@ int32_t moe_route(const void* x, const float* Wr, const float* bias, const moe_c
   if (!ws_ok(workspace, workspace_bytes, moe_route_workspace_bytes(cfg))) return MOE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* status = at<int>(workspace, 0);
-  return cuda_status(launch_router(x, Wr, bias, router_params(*cfg), topk_ids, topk_w,
+  RouterParams rp = router_params(*cfg);
+  rp.mask = token_mask;
+  return cuda_status(launch_router(x, Wr, bias, rp, topk_ids, topk_w,
                                    at<void>(workspace, align_up(sizeof(DevStatus))), status,
                                    DEFAULT_TIMEOUT_NS, s));
+}
+
+int32_t moe_route(const void* x, const float* Wr, const float* bias, const moe_cfg_t* cfg,
+                  int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  return moe_route_masked(x, Wr, bias, nullptr, cfg, topk_ids, topk_w, workspace,
+                          workspace_bytes, stream);
 }
 
 int32_t moe_permute(const int32_t* topk_ids, const float* topk_w, const void* x,

@@ -86,6 +86,7 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity,
 
 struct TileCoord {
   int g, row0, rows, nt;
+  int gstart;  // first row of the group (0 for a single group)
 };
 
 __device__ __forceinline__ TileCoord tile_coord(int tile, const GemmArgs& a, const int* mts,
@@ -97,6 +98,7 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const GemmArgs& a, con
     c.g = 0;
     c.row0 = mt * TILE_M;
     c.rows = min(TILE_M, a.single_rows - c.row0);
+    c.gstart = 0;
     return c;
   }
   int lo = 0, hi = a.num_groups;  // largest g with mts[g] <= mt
@@ -108,6 +110,7 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const GemmArgs& a, con
       hi = mid;
   }
   c.g = lo;
+  c.gstart = rs[lo];
   c.row0 = rs[lo] + (mt - mts[lo]) * TILE_M;
   c.rows = min(TILE_M, rs[lo + 1] - c.row0);
   return c;
@@ -140,7 +143,8 @@ __device__ __forceinline__ RowIn epilogue_row_inputs(const GemmArgs& a, const Ti
       const int row = tc.row0 + r_in_tile;
       if (tc.g == a.alt_group || !a.dest_pos) {  // unweighted rows at t*dest_mul + dest_add
         in.w = 1.0f;
-        in.drow = (row - (tc.g == a.alt_group ? a.alt_row0 : 0)) * a.dest_mul + a.dest_add;
+        // the group's rows are its tokens in order
+        in.drow = (row - (tc.g == a.alt_group ? tc.gstart : 0)) * a.dest_mul + a.dest_add;
       } else {
         in.w = a.row_scale ? a.row_scale[row] : 1.0f;
         in.drow = a.dest_pos[row];
@@ -277,7 +281,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const bool alt = tc.g == args.alt_group;
         const CUtensorMap* ma = alt ? &tmA2 : &tmA;
         const CUtensorMap* mb = alt ? &tmB2 : &tmB;
-        const int a_row = tc.row0 + BM * (int)rank - (alt ? args.alt_row0 : 0);
+        const int a_row = tc.row0 + BM * (int)rank - (alt && args.alt_rebase ? tc.gstart : 0);
         const int b_grp = alt ? 0 : tc.g;
         const int b_row = tc.nt * args.n_out_tile + (int)rank * args.b_second;
         // a CTA whose half of the tile holds no rows of the group skips its A

@@ -89,6 +89,7 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity,
 
 struct Item {
   int g, row0, rows, mt;
+  int gstart;  // first row of the group
 };
 
 template <int CHUNK>
@@ -106,6 +107,7 @@ __device__ __forceinline__ Item item_coord(int item, int n_tiles, int groups, co
       hi = mid;
   }
   it.g = lo;
+  it.gstart = rs[lo];
   it.row0 = rs[lo] + (ch - cs[lo]) * CHUNK;
   it.rows = min(CHUNK, rs[lo + 1] - it.row0);
   return it;
@@ -212,7 +214,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const CUtensorMap* mx = alt ? &tmX2 : &tmX;
         const int w_grp = alt ? 0 : it.g;
         const int w_row = it.mt * args.n_out_tile;
-        const int x_row = it.row0 - (alt ? args.alt_row0 : 0);
+        const int x_row = it.row0 - (alt && args.alt_rebase ? it.gstart : 0);
         const int nb = (it.rows + XBOX - 1) / XBOX;
         const uint32_t tx = S::NW * W_BYTES + nb * XBOX_BYTES;
         for (int ks = 0; ks < args.k_steps; ++ks) {
@@ -312,7 +314,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             int d;
             if (alt || !args.dest_pos) {
               w = 1.0f;
-              d = (row - (alt ? args.alt_row0 : 0)) * args.dest_mul + args.dest_add;
+              d = (row - (alt ? it.gstart : 0)) * args.dest_mul + args.dest_add;
             } else {
               w = args.row_scale ? args.row_scale[row] : 1.0f;
               d = args.dest_pos[row];

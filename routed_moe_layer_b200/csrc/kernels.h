@@ -32,6 +32,7 @@ struct RouterParams {
   int T, H, E, top_k, n_group, topk_group, norm_topk_prob;
   float rsf;
   int clear_status;  // 1: the router's first kernel clears the status word
+  const uint8_t* mask = nullptr;  // [T] or null: 0 = padding token (ids -1, weights 0)
 };
 
 // Router on the tensor cores: scratch holds the 3-term bf16 split of Wr and the
@@ -61,6 +62,7 @@ struct PermuteOut {
                           // (expert_offsets / mtile_start then have E+2 entries)
   float* w_of;          // [T*k] or null
   void* xp;             // [T*k, H] bf16 or null
+  const uint8_t* mask = nullptr;  // [T] or null: tokens with 0 (padding) take no rows
 };
 
 cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const void* x, int T,
@@ -75,8 +77,9 @@ struct GemmArgs {
   const int* row_start;    // [num_groups+1] device first row of each group
   int num_groups;
   int single_rows;         // rows of the only group when mtile_start == null
-  int alt_group;           // group read through the second pair of maps (-1: none); its
-  int alt_row0;            //   rows start at alt_row0 in the first A map's row numbering
+  int alt_group;           // group read through the second pair of maps (-1: none)
+  int alt_rebase;          // 1: its A rows are read at (row - the group's first row),
+                           //    e.g. x for the shared expert; 0: at their own row
   int n_tiles;             // output tiles along N
   int k_steps;             // K / 64
   int n_out_tile;          // output columns per tile: 128 (SwiGLU) or 256

@@ -28,12 +28,13 @@ constexpr int MAXE = 128;
 constexpr int MAX_TOPK_PERMUTE = 16;
 
 __device__ __forceinline__ void build_masks(const int32_t* __restrict__ ids, int T, int E,
-                                            int top_k, uint32_t (*masks)[MAXE], int* status) {
+                                            int top_k, const uint8_t* __restrict__ tmask,
+                                            uint32_t (*masks)[MAXE], int* status) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < PW * MAXE; i += PT) (&masks[0][0])[i] = 0u;
   __syncthreads();
   const int t = blockIdx.x * PT + tid;
-  if (t < T) {
+  if (t < T && (!tmask || tmask[t] != 0)) {  // padding tokens take no rows
     for (int j = 0; j < top_k; ++j) {
       const int e = ids[(size_t)t * top_k + j];
       if (e >= 0 && e < E)
@@ -47,11 +48,12 @@ __device__ __forceinline__ void build_masks(const int32_t* __restrict__ ids, int
 
 __global__ void __launch_bounds__(PT)
     permute_count_kernel(const int32_t* __restrict__ ids, int T, int E, int top_k,
-                         int* __restrict__ blk_hist, int* status) {
+                         const uint8_t* __restrict__ tmask, int* __restrict__ blk_hist,
+                         int* status) {
   __shared__ uint32_t masks[PW][MAXE];
   pdl_launch_dependents();
   pdl_wait();
-  build_masks(ids, T, E, top_k, masks, status);
+  build_masks(ids, T, E, top_k, tmask, masks, status);
   for (int e = threadIdx.x; e < E; e += PT) {
     int cnt = 0;
 #pragma unroll
@@ -173,7 +175,8 @@ __global__ void __launch_bounds__(1024)
                          int E, int top_k, int extra_rows, int* __restrict__ expert_offsets,
                          int* __restrict__ mtile_start, int* __restrict__ row_of,
                          int* __restrict__ tok_of, float* __restrict__ w_of,
-                         int* __restrict__ pos_of, int slot_stride, int* status) {
+                         int* __restrict__ pos_of, int slot_stride,
+                         const uint8_t* __restrict__ tmask, int* status) {
   __shared__ uint32_t masks[32][MAXE];
   __shared__ int wbase[32][MAXE];
   __shared__ int tot[MAXE];
@@ -185,11 +188,12 @@ __global__ void __launch_bounds__(1024)
   for (int i = tid; i < 32 * MAXE; i += 1024) (&masks[0][0])[i] = 0u;
   __syncthreads();
   const int t = tid;
+  const bool real = t < T && (!tmask || tmask[t] != 0);  // padding tokens take no rows
   int my_e[MAX_TOPK_PERMUTE];
 #pragma unroll
   for (int j = 0; j < MAX_TOPK_PERMUTE; ++j) {
     my_e[j] = -1;
-    if (t < T && j < top_k) {
+    if (real && j < top_k) {
       const int e = ids[(size_t)t * top_k + j];
       if (e >= 0 && e < E) {
         my_e[j] = e;
@@ -236,12 +240,12 @@ __global__ void __launch_bounds__(PT)
                            int T, int E, int top_k, const int* __restrict__ blk_base,
                            int* __restrict__ row_of, int* __restrict__ tok_of,
                            float* __restrict__ w_of, int* __restrict__ pos_of, int slot_stride,
-                           int* status) {
+                           const uint8_t* __restrict__ tmask, int* status) {
   __shared__ uint32_t masks[PW][MAXE];
   __shared__ int wbase[PW][MAXE];
   pdl_launch_dependents();
   pdl_wait();
-  build_masks(ids, T, E, top_k, masks, status);
+  build_masks(ids, T, E, top_k, tmask, masks, status);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int e = tid; e < E; e += PT) {
     int run = blk_base[(size_t)blockIdx.x * E + e];
@@ -254,10 +258,11 @@ __global__ void __launch_bounds__(PT)
   __syncthreads();
   const int t = blockIdx.x * PT + tid;
   if (t >= T) return;
+  const bool pad = tmask && tmask[t] == 0;
   const uint32_t lower = (1u << lane) - 1u;
   for (int j = 0; j < top_k; ++j) {
     const size_t tj = (size_t)t * top_k + j;
-    const int e = ids[tj];
+    const int e = pad ? -1 : ids[tj];
     if (e < 0 || e >= E) {
       row_of[tj] = -1;
       continue;
@@ -314,20 +319,20 @@ cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const v
   if (T <= PERMUTE_SMALL_T) {
     err = launch_chained(permute_small_kernel, dim3(1), dim3(1024), 0, stream, topk_ids, topk_w, T,
                          E, top_k, o.extra_rows, o.expert_offsets, o.mtile_start, o.row_of,
-                         o.tok_of, o.w_of, o.pos_of, o.slot_stride, o.status);
+                         o.tok_of, o.w_of, o.pos_of, o.slot_stride, o.mask, o.status);
     if (err != cudaSuccess) return err;
     return launch_gather(x, T, H, top_k, o, stream);
   }
   const int nblk = (T + PT - 1) / PT;
-  err = launch_chained(permute_count_kernel, dim3(nblk), dim3(PT), 0, stream, topk_ids,
-                                   T, E, top_k, o.blk_hist, o.status);
+  err = launch_chained(permute_count_kernel, dim3(nblk), dim3(PT), 0, stream, topk_ids, T, E,
+                       top_k, o.mask, o.blk_hist, o.status);
   if (err != cudaSuccess) return err;
   err = launch_chained(permute_scan_kernel, dim3(1), dim3(1024), 0, stream, o.blk_hist, nblk, E,
                        o.extra_rows, o.expert_offsets, o.mtile_start);
   if (err != cudaSuccess) return err;
   err = launch_chained(permute_scatter_kernel, dim3(nblk), dim3(PT), 0, stream, topk_ids, topk_w,
                        T, E, top_k, (const int*)o.blk_hist, o.row_of, o.tok_of, o.w_of, o.pos_of,
-                       o.slot_stride, o.status);
+                       o.slot_stride, o.mask, o.status);
   if (err != cudaSuccess) return err;
   return launch_gather(x, T, H, top_k, o, stream);
 }

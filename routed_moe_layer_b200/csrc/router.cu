@@ -385,7 +385,11 @@ __global__ void __launch_bounds__(SEL_WARPS * 32)
       }
     }
     if (tok_ok && sl < p.top_k) {
-      const float wv = p.norm_topk_prob ? p.rsf * (my_s / sum) : p.rsf * my_s;
+      float wv = p.norm_topk_prob ? p.rsf * (my_s / sum) : p.rsf * my_s;
+      if (p.mask && p.mask[t] == 0) {  // padding token: no routed expert
+        my_id = -1;
+        wv = 0.f;
+      }
       topk_ids[(size_t)t * p.top_k + sl] = my_id;
       topk_w[(size_t)t * p.top_k + sl] = wv;
     }

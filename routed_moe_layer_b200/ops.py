@@ -42,7 +42,7 @@ class MoeForwardOpts(ctypes.Structure):
     _fields_ = [
         ("residual", ctypes.c_void_p), ("topk_ids", ctypes.c_void_p),
         ("topk_w", ctypes.c_void_p), ("stage_events", ctypes.POINTER(ctypes.c_void_p)),
-        ("wait_timeout_ns", ctypes.c_int64),
+        ("wait_timeout_ns", ctypes.c_int64), ("token_mask", ctypes.c_void_p),
     ]
 
 
@@ -91,6 +91,7 @@ def lib() -> ctypes.CDLL:
         "moe_permute_workspace_bytes": (sz, [cfgp]),
         "moe_workspace_bytes": (sz, [cfgp]),
         "moe_route": (i32, [vp, vp, vp, cfgp, vp, vp, vp, sz, vp]),
+        "moe_route_masked": (i32, [vp, vp, vp, vp, cfgp, vp, vp, vp, sz, vp]),
         "moe_permute": (i32, [vp, vp, vp, cfgp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "moe_forward": (i32, [vp, vp, vp, vp, vp, vp, vp, cfgp, vp,
                               ctypes.POINTER(MoeForwardOpts), vp, sz, vp]),
@@ -159,18 +160,27 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def route(x: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor, cfg: BlockConfig):
-    """Router: returns (topk_ids int32 [T,k], topk_w fp32 [T,k])."""
+def route(x: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor, cfg: BlockConfig,
+          token_mask: Optional[torch.Tensor] = None):
+    """Router: returns (topk_ids int32 [T,k], topk_w fp32 [T,k]); with a uint8
+    token_mask [T], padding tokens (0) get ids -1 and weights 0."""
     T, H = cfg.T, cfg.H
     _need(x, "x", torch.bfloat16, (T, H))
     _need(Wr, "Wr", torch.float32, (cfg.E, H))
     _need(bias, "bias", torch.float32, (cfg.E,))
+    if token_mask is not None:
+        _need(token_mask, "token_mask", torch.uint8, (T,))
     ids = torch.empty((T, cfg.top_k), dtype=torch.int32, device=x.device)
     w = torch.empty((T, cfg.top_k), dtype=torch.float32, device=x.device)
     c = cfg.c()
     ws = alloc_workspace(lib().moe_route_workspace_bytes(ctypes.byref(c)), x.device)
-    _check(lib().moe_route(_ptr(x), _ptr(Wr), _ptr(bias), ctypes.byref(c), _ptr(ids), _ptr(w),
-                           _ptr(ws), ws.numel(), _stream_ptr()), "moe_route")
+    if token_mask is None:
+        _check(lib().moe_route(_ptr(x), _ptr(Wr), _ptr(bias), ctypes.byref(c), _ptr(ids),
+                               _ptr(w), _ptr(ws), ws.numel(), _stream_ptr()), "moe_route")
+    else:
+        _check(lib().moe_route_masked(_ptr(x), _ptr(Wr), _ptr(bias), _ptr(token_mask),
+                                      ctypes.byref(c), _ptr(ids), _ptr(w), _ptr(ws), ws.numel(),
+                                      _stream_ptr()), "moe_route_masked")
     return ids, w
 
 
@@ -232,8 +242,10 @@ def forward(x: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor, w13: torch.Te
             cfg: BlockConfig, residual: Optional[torch.Tensor] = None,
             out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
             topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
-            timer: Optional[StageTimer] = None, wait_timeout_ns: int = 0) -> torch.Tensor:
-    """Block forward; returns out bf16 [T,H] (written in place when ``out`` is given)."""
+            timer: Optional[StageTimer] = None, wait_timeout_ns: int = 0,
+            token_mask: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Block forward; returns out bf16 [T,H] (written in place when ``out`` is given).
+    token_mask: uint8 [T] padding mask (0 = padding: shared expert only)."""
     T, H, E, I, Is, k = cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared, cfg.top_k
     _need(x, "x", torch.bfloat16, (T, H))
     _need(Wr, "Wr", torch.float32, (E, H))
@@ -253,6 +265,8 @@ def forward(x: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor, w13: torch.Te
         _need(topk_ids, "topk_ids", torch.int32, (T, k))
     if topk_w is not None:
         _need(topk_w, "topk_w", torch.float32, (T, k))
+    if token_mask is not None:
+        _need(token_mask, "token_mask", torch.uint8, (T,))
     if workspace is None:
         workspace = alloc_workspace(workspace_bytes(cfg), x.device)
     opts = MoeForwardOpts(
@@ -260,7 +274,8 @@ def forward(x: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor, w13: torch.Te
         topk_ids=None if topk_ids is None else topk_ids.data_ptr(),
         topk_w=None if topk_w is None else topk_w.data_ptr(),
         stage_events=timer.as_ptr() if timer is not None else None,
-        wait_timeout_ns=int(wait_timeout_ns))
+        wait_timeout_ns=int(wait_timeout_ns),
+        token_mask=None if token_mask is None else token_mask.data_ptr())
     c = cfg.c()
     _check(lib().moe_forward(_ptr(x), _ptr(Wr), _ptr(bias), _ptr(w13), _ptr(w2), _ptr(ws13),
                              _ptr(ws2), ctypes.byref(c), _ptr(out), ctypes.byref(opts),

@@ -38,8 +38,9 @@ def np_inputs(d: dict) -> dict:
 
 
 def check_routing(ids_gpu: torch.Tensor, w_gpu: torch.Tensor, xn, Wrn, biasn, cfg: BlockConfig,
-                  rows=None):
-    """Gate the GPU routing against the oracle; returns a small report."""
+                  rows=None, token_mask=None):
+    """Gate the GPU routing against the oracle; returns a small report.  With a
+    token mask, padding tokens must have ids -1 and weights 0 exactly."""
     ocfg = oracle_cfg(cfg)
     if rows is not None:
         xn = xn[rows]
@@ -48,6 +49,10 @@ def check_routing(ids_gpu: torch.Tensor, w_gpu: torch.Tensor, xn, Wrn, biasn, cf
     wg = w_gpu.cpu().numpy().astype(np.float64)
     if rows is not None:
         ig, wg = ig[rows], wg[rows]
+    if token_mask is not None:
+        pad = np.asarray(token_mask).reshape(-1) == 0
+        assert np.all(ig[pad] == -1) and np.all(wg[pad] == 0.0)
+        ig, wg, ids_ref, w_ref, margin = ig[~pad], wg[~pad], ids_ref[~pad], w_ref[~pad], margin[~pad]
     far = margin > TIE_MARGIN
     og = np.argsort(ig, axis=1)
     orf = np.argsort(ids_ref, axis=1)
@@ -67,7 +72,7 @@ def check_routing(ids_gpu: torch.Tensor, w_gpu: torch.Tensor, xn, Wrn, biasn, cf
 
 
 def check_output(out_gpu: torch.Tensor, ids_gpu: torch.Tensor, d_np: dict, cfg: BlockConfig,
-                 tokens=None, residual_np=None):
+                 tokens=None, residual_np=None, token_mask=None):
     """Gate the GPU output against the float64 oracle under the GPU's expert
     choice, on all tokens or on the given token sample."""
     ocfg = oracle_cfg(cfg)
@@ -75,11 +80,13 @@ def check_output(out_gpu: torch.Tensor, ids_gpu: torch.Tensor, d_np: dict, cfg: 
     args = (d_np["x"], d_np["Wr"], d_np["bias"], d_np["w13"], d_np["w2"],
             d_np.get("ws13"), d_np.get("ws2"), ocfg)
     if tokens is None:
-        ref, _, _, _ = oracle.moe_forward(*args, residual=residual_np, ids=ids)
+        ref, _, _, _ = oracle.moe_forward(*args, residual=residual_np, ids=ids,
+                                          token_mask=token_mask)
         got = to_np(out_gpu).astype(np.float64)
     else:
         tokens = np.asarray(tokens)
-        ref, _, _, _ = oracle.moe_forward_tokens(tokens, *args, residual=residual_np, ids=ids)
+        ref, _, _, _ = oracle.moe_forward_tokens(tokens, *args, residual=residual_np, ids=ids,
+                                                 token_mask=token_mask)
         got = to_np(out_gpu[torch.as_tensor(tokens, device=out_gpu.device)]).astype(np.float64)
     err = np.abs(got - ref)
     bound = OUT_RTOL * (1.0 + np.abs(ref))

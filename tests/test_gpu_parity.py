@@ -210,6 +210,51 @@ def test_forward_hot_experts_many_tiles(T):
     assert rep["rms_rel"] < 1e-2, rep
 
 
+@pytest.mark.parametrize("T", [300, 1000, 2048])
+def test_forward_padding_mask(T):
+    """Padding tokens (mask 0) take no routed expert and keep the shared
+    expert and the residual; real tokens give bit for bit the unmasked output.
+    T = 300 / 1000 run the swapped GEMMs (32 / 128-row chunks), 2048 the tiled."""
+    H = 512
+    cfg = BlockConfig(T=T, H=H, I=256, I_shared=256)
+    d = inputs.make_block_inputs(T, H, seed=60 + T, I=256, I_shared=256, unit_scale=True)
+    dd = _dev(d)
+    g = torch.Generator().manual_seed(T)
+    mask = (torch.rand(T, generator=g) > 0.2).to(torch.uint8)
+    mask[-37:] = 0  # a padded tail, as in a varlen batch
+    res = torch.randn((T, H), generator=g).to(torch.bfloat16)
+    ref_out, ref_ids, _ = _run(dd, cfg, residual=res.to(DEV))
+    ids = torch.empty((T, cfg.top_k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, cfg.top_k), dtype=torch.float32, device=DEV)
+    ws = ops.alloc_workspace(ops.workspace_bytes(cfg), DEV)
+    out = ops.forward(dd["x"], dd["Wr"], dd["bias"], dd["w13"], dd["w2"], dd["ws13"], dd["ws2"],
+                      cfg, residual=res.to(DEV), workspace=ws, topk_ids=ids, topk_w=w,
+                      token_mask=mask.to(DEV))
+    torch.cuda.synchronize()
+    code, site = ops.read_device_status(ws)
+    assert code == 0, (ops.status_string(code), site)
+    real = mask.bool().to(DEV)
+    assert torch.equal(out[real], ref_out[real]) and torch.equal(ids[real], ref_ids[real])
+    dn = parity.np_inputs(d)
+    parity.check_routing(ids, w, dn["x"], dn["Wr"], dn["bias"], cfg, token_mask=mask.numpy())
+    rep = parity.check_output(out, ids, dn, cfg, residual_np=parity.to_np(res),
+                              token_mask=mask.numpy())
+    assert rep["rms_rel"] < 1e-2, rep
+    # the router alone, and the extremes: every token padding / none
+    ids_r, w_r = ops.route(dd["x"], dd["Wr"], dd["bias"], cfg, token_mask=mask.to(DEV))
+    assert torch.equal(ids_r, ids) and torch.equal(w_r, w)
+    none = torch.zeros(T, dtype=torch.uint8, device=DEV)
+    out0 = ops.forward(dd["x"], dd["Wr"], dd["bias"], dd["w13"], dd["w2"], dd["ws13"], dd["ws2"],
+                       cfg, token_mask=none)
+    torch.cuda.synchronize()
+    parity.check_output(out0, torch.full((T, cfg.top_k), -1, dtype=torch.int32), dn, cfg,
+                        token_mask=np.zeros(T, dtype=np.uint8))
+    all_real = torch.ones(T, dtype=torch.uint8, device=DEV)
+    out1 = ops.forward(dd["x"], dd["Wr"], dd["bias"], dd["w13"], dd["w2"], dd["ws13"], dd["ws2"],
+                       cfg, residual=res.to(DEV), token_mask=all_real)
+    assert torch.equal(out1, ref_out)
+
+
 def test_swapped_and_tiled_gemms_agree():
     """The same tokens through the swapped GEMMs (a small batch) and through
     the 256-row tiles (inside a large batch) give the same bits: both add the
