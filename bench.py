@@ -171,6 +171,8 @@ def cpu_oracle_sample(cfg_id: int, target_s: float = 12.0, d_cpu=None):
         d_cpu = inputs.workload_inputs(cfg_id)
     dn = parity.np_inputs(d_cpu)
     ocfg = parity.oracle_cfg(cfg)
+    m = inputs.token_mask(wl)
+    mask_np = None if m is None else m.numpy()
     rng = np.random.default_rng(0)
     n = 16
     t_used = 0.0
@@ -179,7 +181,7 @@ def cpu_oracle_sample(cfg_id: int, target_s: float = 12.0, d_cpu=None):
         toks = rng.choice(wl.T, n, replace=False)
         t0 = time.perf_counter()
         oracle.moe_forward_tokens(toks, dn["x"], dn["Wr"], dn["bias"], dn["w13"], dn["w2"],
-                                  dn["ws13"], dn["ws2"], ocfg)
+                                  dn["ws13"], dn["ws2"], ocfg, token_mask=mask_np)
         dt = time.perf_counter() - t0
         t_used += dt
         done += n
@@ -208,16 +210,18 @@ def run_reference(args, world, rank):
     dn = parity.np_inputs(d_cpu)
     ocfg = parity.oracle_cfg(cfg)
     per_step = max(1, min(wl.T, args.ref_tokens))
+    m = inputs.token_mask(wl)
+    mask_np = None if m is None else m.numpy()
     rng = np.random.default_rng(1)
     for _ in range(args.warmup if args.ref_warmup else 0):
         toks = rng.choice(wl.T, per_step, replace=False)
         oracle.moe_forward_tokens(toks, dn["x"], dn["Wr"], dn["bias"], dn["w13"], dn["w2"],
-                                  dn["ws13"], dn["ws2"], ocfg)
+                                  dn["ws13"], dn["ws2"], ocfg, token_mask=mask_np)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         toks = rng.choice(wl.T, per_step, replace=False)
         oracle.moe_forward_tokens(toks, dn["x"], dn["Wr"], dn["bias"], dn["w13"], dn["w2"],
-                                  dn["ws13"], dn["ws2"], ocfg)
+                                  dn["ws13"], dn["ws2"], ocfg, token_mask=mask_np)
     dt = time.perf_counter() - t0
     tps = per_step * args.steps / dt
     try:
@@ -265,11 +269,14 @@ def run_ours(args, world, rank, local):
     xn_buf = torch.empty_like(x)
     ids = torch.empty((wl.T, cfg.top_k), dtype=torch.int32, device=dev)
 
+    mask_dev = inputs.token_mask(wl, dev)  # padding mask of the workload, or None
+
     def step(xin, timer=None):
         if layers == 1:
             w = weights[0]
             return ops.forward(xin, w["Wr"], w["bias"], w["w13"], w["w2"], w["ws13"], w["ws2"],
-                               cfg, out=out, workspace=ws, timer=timer, topk_ids=ids)
+                               cfg, out=out, workspace=ws, timer=timer, topk_ids=ids,
+                               token_mask=mask_dev)
         # residual stack: x <- x + block_l(RMSNorm(x)), updated in place in `out`
         out.copy_(xin)
         for l, w in enumerate(weights):
@@ -316,7 +323,8 @@ def run_ours(args, world, rank, local):
         step(x, timer=t)
     torch.cuda.synchronize()
     per_stage = {k: float(np.mean([t.stage_ms()[k] for t in split_timers])) for k in ops.STAGES}
-    counts = torch.bincount(ids.reshape(-1).long(), minlength=cfg.E)
+    flat = ids.reshape(-1).long()
+    counts = torch.bincount(flat[flat >= 0], minlength=cfg.E)  # padding tokens have ids -1
     experts_used = int((counts > 0).sum().item())
 
     # end to end: pinned host tokens -> device -> block -> host, every step.
@@ -341,7 +349,7 @@ def run_ours(args, world, rank, local):
     _barrier(world)
     e2e_serial_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     e2e_ms, e2e_mode = e2e_serial_ms, "serial: copy in, block, copy out, one batch at a time"
-    if layers == 1:
+    if layers == 1 and mask_dev is None:
         # the library's host-batch entry point: every step's batch is copied in
         # and its output copied out, the copies of the neighbouring batches
         # overlapping each batch's kernels (two copy streams)
@@ -374,10 +382,15 @@ def run_ours(args, world, rank, local):
         total_tokens = tok_per_step * world
         value = total_tokens / (ms * 1e-3)
         fpt = flops_per_token(cfg)
-        tflops = value * fpt / 1e12
+        # padding tokens (token mask 0) run only the router and the shared expert
+        n_pad = 0 if mask_dev is None else int((mask_dev == 0).sum().item())
+        n_real = wl.T - n_pad
+        fpt_pad = 2.0 * cfg.E * cfg.H + 6.0 * cfg.H * cfg.I_shared
+        flops_per_step = n_real * fpt + n_pad * fpt_pad  # one layer, one rank
+        tflops = flops_per_step * layers * world / (ms * 1e-3) / 1e12
         # the expert-up launch also runs the shared expert as one more group
         # when its intermediate size equals the experts' (the model's case)
-        R = wl.T * cfg.top_k
+        R = n_real * cfg.top_k
         up_rows = R + (wl.T if cfg.I_shared == cfg.I else 0)
         up_flops = 2.0 * up_rows * cfg.H * (2 * cfg.I)
         up_ms = up_ms_live
@@ -389,15 +402,31 @@ def run_ours(args, world, rank, local):
         achieved = up_flops / (up_ms * 1e-3) / 1e12
         layer_ms = ms / layers
         hbm_bytes = algorithmic_bytes(cfg, experts_used)
-        rf = {"bound": "tensor",
-              "kernel": "grouped_gemm_kernel<SwiGLU> (expert up, shared expert folded in)",
-              "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
-              "frac": achieved / peak_tf,
-              "peak_source": f"{peak_src} bf16 dense {'sustained' if long_region else 'burst'}",
-              "traffic": measured_traffic("grouped_gemm_kernel<EPI_SWIGLU>", wl.name),
-              "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
-              "layer_roofline_frac": max(fpt * wl.T / peak_tf / 1e12,
-                                         hbm_bytes / peaks["hbm_gbs"] / 1e9) / (layer_ms * 1e-3)}
+        t_flop = flops_per_step / peak_tf / 1e12
+        t_hbm = hbm_bytes / peaks["hbm_gbs"] / 1e9
+        swapped = wl.T * cfg.top_k <= 64 * cfg.E  # the kernel the library picks for this shape
+        kernel = ("grouped_gemm_swap_kernel<SwiGLU> (expert up, shared expert folded in)"
+                  if swapped else
+                  "grouped_gemm_kernel<SwiGLU> (expert up, shared expert folded in)")
+        if t_hbm > t_flop:
+            # HBM-bound layer: the expert-up launch streams w13 of the used experts and
+            # ws13, reads the gathered rows and x, writes h
+            up_bytes = (experts_used * 2.0 * cfg.I * cfg.H * 2 + 2.0 * cfg.I_shared * cfg.H * 2 +
+                        up_rows * cfg.H * 2 + up_rows * cfg.I * 2)
+            ach = up_bytes / (up_ms * 1e-3) / 1e9
+            rf = {"bound": "hbm", "kernel": kernel, "achieved": ach, "peak": peaks["hbm_gbs"],
+                  "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+                  "peak_source": f"{peak_src} HBM copy bandwidth",
+                  "algorithmic_bytes_per_launch": up_bytes, "flops_per_launch": up_flops}
+        else:
+            rf = {"bound": "tensor", "kernel": kernel,
+                  "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                  "frac": achieved / peak_tf,
+                  "peak_source": f"{peak_src} bf16 dense {'sustained' if long_region else 'burst'}"}
+        rf["traffic"] = (None if swapped else
+                         measured_traffic("grouped_gemm_kernel<EPI_SWIGLU>", wl.name))
+        rf["traffic_unit"] = "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
+        rf["layer_roofline_frac"] = max(t_flop, t_hbm) / (layer_ms * 1e-3)
         cpu_tps, cores, sample = (None, None, None)
         if world == 1 and not args.no_cpu_baseline:
             cpu_tps, cores, sample = cpu_oracle_sample(args.config, target_s=args.cpu_seconds)
@@ -410,6 +439,7 @@ def run_ours(args, world, rank, local):
                        "I_shared": cfg.I_shared, "top_k": cfg.top_k, "n_group": cfg.n_group,
                        "topk_group": cfg.topk_group, "layers": layers,
                        "tokens_per_gpu_per_step": tok_per_step,
+                       "padding_tokens_per_layer": n_pad,
                        "l2": "inputs larger than L2: 1.2 GB of expert weights read per layer"},
             "tflops": tflops,
             "roofline": rf,

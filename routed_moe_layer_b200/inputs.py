@@ -30,6 +30,8 @@ import torch
 #   2: one layer, 19412 tokens (18900 video = 21 x 30x30 + 512 text), H=2048
 #   3: CFG batch 2 x 19412 = 38824 rows, H=2048, bias +0.5 on 8 hot experts
 #   4: 48 residual layers x (RMSNorm -> block) at 19412 tokens, H=2048
+#   5: CFG batch 2 x 19412 rows with padded text: the second prompt has 64 real
+#      text tokens, its other 448 text rows are padding (token mask 0)
 HOT_EXPERTS = tuple(range(0, 128, 16))  # two per group of 32
 
 
@@ -42,6 +44,7 @@ class Workload:
     layers: int = 1
     hot_experts: Optional[Sequence[int]] = None
     hot_bias: float = 0.5
+    padding: Optional[Sequence[tuple]] = None  # [start, stop) row ranges of padding tokens
 
 
 WORKLOADS = {
@@ -50,7 +53,19 @@ WORKLOADS = {
     2: Workload("moe_layer_T19412_H2048", 19412, 2048, 2),
     3: Workload("moe_layer_cfg2x19412_H2048_skewed", 38824, 2048, 3, hot_experts=HOT_EXPERTS),
     4: Workload("moe_stack48_T19412_H2048", 19412, 2048, 4, layers=48),
+    5: Workload("moe_layer_cfg2x19412_H2048_padded", 38824, 2048, 5,
+                padding=((19412 + 18900 + 64, 38824),)),
 }
+
+
+def token_mask(w: Workload, device="cpu") -> Optional[torch.Tensor]:
+    """uint8 [T] mask of a workload (1 = real token, 0 = padding), or None."""
+    if not w.padding:
+        return None
+    m = torch.ones(w.T, dtype=torch.uint8)
+    for a, b in w.padding:
+        m[a:b] = 0
+    return m.to(device)
 
 
 def _gen(seed: int, device) -> torch.Generator:

@@ -24,12 +24,13 @@ def _dev(d):
     return {k: (None if v is None else v.to(DEV)) for k, v in d.items()}
 
 
-def _run(d, cfg, residual=None):
+def _run(d, cfg, residual=None, token_mask=None):
     ids = torch.empty((cfg.T, cfg.top_k), dtype=torch.int32, device=DEV)
     w = torch.empty((cfg.T, cfg.top_k), dtype=torch.float32, device=DEV)
     ws = ops.alloc_workspace(ops.workspace_bytes(cfg), DEV)
     out = ops.forward(d["x"], d["Wr"], d["bias"], d["w13"], d["w2"], d.get("ws13"), d.get("ws2"),
-                      cfg, residual=residual, workspace=ws, topk_ids=ids, topk_w=w)
+                      cfg, residual=residual, workspace=ws, topk_ids=ids, topk_w=w,
+                      token_mask=token_mask)
     torch.cuda.synchronize()
     code, site = ops.read_device_status(ws)
     assert code == 0, (ops.status_string(code), site)
@@ -283,18 +284,21 @@ def test_forward_small_workloads_in_full(wid):
     assert orep["rms_rel"] < 1e-2
 
 
-@pytest.mark.parametrize("wid", [2, 3])
+@pytest.mark.parametrize("wid", [2, 3, 5])
 def test_forward_large_workloads_sampled(wid):
     wl = inputs.WORKLOADS[wid]
     cfg = BlockConfig(T=wl.T, H=wl.H)
     d = inputs.workload_inputs(wid)
-    out, ids, w = _run(_dev(d), cfg)
+    mask = inputs.token_mask(wl)
+    mask_np = None if mask is None else mask.numpy()
+    out, ids, w = _run(_dev(d), cfg, token_mask=None if mask is None else mask.to(DEV))
     dn = parity.np_inputs(d)
-    rrep = parity.check_routing(ids, w, dn["x"], dn["Wr"], dn["bias"], cfg)
+    rrep = parity.check_routing(ids, w, dn["x"], dn["Wr"], dn["bias"], cfg, token_mask=mask_np)
     rng = np.random.default_rng(wid)
-    sample = np.concatenate([[0, wl.T - 1], rng.choice(wl.T, 254, replace=False)])
-    orep = parity.check_output(out, ids, dn, cfg, tokens=sample)
-    counts = np.bincount(ids.cpu().numpy().ravel(), minlength=128)
+    sample = np.concatenate([[0, wl.T - 1, wl.T - 441], rng.choice(wl.T, 253, replace=False)])
+    orep = parity.check_output(out, ids, dn, cfg, tokens=sample, token_mask=mask_np)
+    ids_np = ids.cpu().numpy()
+    counts = np.bincount(ids_np[ids_np >= 0].ravel(), minlength=128)
     print(f"{wl.name}: routing {rrep} output {orep} rows/expert min {counts.min()} "
           f"max {counts.max()}")
     assert orep["rms_rel"] < 1e-2
