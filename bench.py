@@ -56,6 +56,20 @@ def algorithmic_bytes(cfg: BlockConfig, experts_used: int) -> float:
             cfg.E * 4 + 2.0 * cfg.T * cfg.H * 2)
 
 
+class CallTimer:
+    """Two CUDA events around one call on the current stream (created and
+    recorded once up front so that their handles exist)."""
+
+    def __init__(self):
+        self.begin = torch.cuda.Event(enable_timing=True)
+        self.end = torch.cuda.Event(enable_timing=True)
+        self.begin.record()
+        self.end.record()
+
+    def stage_ms(self):
+        return {"expert_up": self.begin.elapsed_time(self.end)}
+
+
 def measured_traffic(kernel: str, workload: str):
     """DRAM bytes per launch of ``kernel`` from the committed ncu summary, or None when the
     kernel's source has changed since the counters were taken (or none were taken)."""
@@ -180,8 +194,11 @@ def cpu_oracle_sample(cfg_id: int, target_s: float = 12.0, d_cpu=None):
     while True:
         toks = rng.choice(wl.T, n, replace=False)
         t0 = time.perf_counter()
-        oracle.moe_forward_tokens(toks, dn["x"], dn["Wr"], dn["bias"], dn["w13"], dn["w2"],
-                                  dn["ws13"], dn["ws2"], ocfg, token_mask=mask_np)
+        if wl.dense_I:
+            oracle.dense_ffn(dn["x"][toks], dn["w13"], dn["w2"])
+        else:
+            oracle.moe_forward_tokens(toks, dn["x"], dn["Wr"], dn["bias"], dn["w13"], dn["w2"],
+                                      dn["ws13"], dn["ws2"], ocfg, token_mask=mask_np)
         dt = time.perf_counter() - t0
         t_used += dt
         done += n
@@ -213,15 +230,18 @@ def run_reference(args, world, rank):
     m = inputs.token_mask(wl)
     mask_np = None if m is None else m.numpy()
     rng = np.random.default_rng(1)
+    def one(toks):
+        if wl.dense_I:
+            oracle.dense_ffn(dn["x"][toks], dn["w13"], dn["w2"])
+        else:
+            oracle.moe_forward_tokens(toks, dn["x"], dn["Wr"], dn["bias"], dn["w13"], dn["w2"],
+                                      dn["ws13"], dn["ws2"], ocfg, token_mask=mask_np)
+
     for _ in range(args.warmup if args.ref_warmup else 0):
-        toks = rng.choice(wl.T, per_step, replace=False)
-        oracle.moe_forward_tokens(toks, dn["x"], dn["Wr"], dn["bias"], dn["w13"], dn["w2"],
-                                  dn["ws13"], dn["ws2"], ocfg, token_mask=mask_np)
+        one(rng.choice(wl.T, per_step, replace=False))
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        toks = rng.choice(wl.T, per_step, replace=False)
-        oracle.moe_forward_tokens(toks, dn["x"], dn["Wr"], dn["bias"], dn["w13"], dn["w2"],
-                                  dn["ws13"], dn["ws2"], ocfg, token_mask=mask_np)
+        one(rng.choice(wl.T, per_step, replace=False))
     dt = time.perf_counter() - t0
     tps = per_step * args.steps / dt
     try:
@@ -236,7 +256,7 @@ def run_reference(args, world, rank):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": 128, "I": 768,
                    "top_k": 8, "tokens_per_step_sampled": per_step},
-        "tflops": tps * flops_per_token(cfg) / 1e12,
+        "tflops": tps * (6.0 * wl.H * wl.dense_I if wl.dense_I else flops_per_token(cfg)) / 1e12,
         "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
                          "sample": f"{per_step} random tokens of {wl.name} per step"},
         "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -257,14 +277,19 @@ def run_ours(args, world, rank, local):
     layers = wl.layers
     # weights: identical on every rank; tokens: a different batch per rank
     gen_dev = dev if layers > 1 else "cpu"
+    dense = wl.dense_I > 0  # a dense feed-forward layer instead of the MoE block
     weights = []
     for l in range(layers):
-        wd = inputs.make_weights(wl.H, wl.seed, device=gen_dev, layer=l,
-                                 hot_experts=wl.hot_experts, hot_bias=wl.hot_bias)
+        if dense:
+            wd = inputs.make_dense_weights(wl.H, wl.dense_I, wl.seed, device=gen_dev)
+        else:
+            wd = inputs.make_weights(wl.H, wl.seed, device=gen_dev, layer=l,
+                                     hot_experts=wl.hot_experts, hot_bias=wl.hot_bias)
         weights.append({k: (None if v is None else v.to(dev)) for k, v in wd.items()})
     x_host = inputs.make_tokens(wl.T, wl.H, rank_token_seed(wl.seed, rank)).pin_memory()
     x = x_host.to(dev)
-    ws = ops.alloc_workspace(ops.workspace_bytes(cfg), dev)
+    ws = ops.alloc_workspace(ops.workspace_bytes(cfg) if not dense else
+                             ops.lib().moe_dense_ffn_workspace_bytes(wl.T, wl.H, wl.dense_I), dev)
     out = torch.empty_like(x)
     xn_buf = torch.empty_like(x)
     ids = torch.empty((wl.T, cfg.top_k), dtype=torch.int32, device=dev)
@@ -272,6 +297,14 @@ def run_ours(args, world, rank, local):
     mask_dev = inputs.token_mask(wl, dev)  # padding mask of the workload, or None
 
     def step(xin, timer=None):
+        if dense:  # the whole layer is timed: both GEMMs (no stage events inside)
+            w = weights[0]
+            if timer is not None:
+                timer.begin.record(torch.cuda.current_stream())
+            ops.dense_ffn(xin, w["w13"], w["w2"], out=out, workspace=ws)
+            if timer is not None:
+                timer.end.record(torch.cuda.current_stream())
+            return out
         if layers == 1:
             w = weights[0]
             return ops.forward(xin, w["Wr"], w["bias"], w["w13"], w["w2"], w["ws13"], w["ws2"],
@@ -296,7 +329,8 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream()
     # only the dominant kernel is timed inside the headline region: every
     # recorded event orders the chained kernels around it
-    timers = [ops.StageTimer(stages=("expert_up",)) for _ in range(args.steps)]
+    timers = [(CallTimer() if dense else ops.StageTimer(stages=("expert_up",)))
+              for _ in range(args.steps)]
     sampler = ClockSampler(local)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(world)
@@ -318,14 +352,19 @@ def run_ours(args, world, rank, local):
     # the expert-up stage is exactly one kernel launch
     up_ms_live = float(np.mean([t.stage_ms()["expert_up"] for t in timers]))
     # stage split, from a separate pass with every stage boundary recorded
-    split_timers = [ops.StageTimer() for _ in range(min(args.steps, 10))]
-    for t in split_timers:
-        step(x, timer=t)
-    torch.cuda.synchronize()
-    per_stage = {k: float(np.mean([t.stage_ms()[k] for t in split_timers])) for k in ops.STAGES}
-    flat = ids.reshape(-1).long()
-    counts = torch.bincount(flat[flat >= 0], minlength=cfg.E)  # padding tokens have ids -1
-    experts_used = int((counts > 0).sum().item())
+    if dense:
+        per_stage = {"dense_ffn": up_ms_live}
+        experts_used = 0
+    else:
+        split_timers = [ops.StageTimer() for _ in range(min(args.steps, 10))]
+        for t in split_timers:
+            step(x, timer=t)
+        torch.cuda.synchronize()
+        per_stage = {k: float(np.mean([t.stage_ms()[k] for t in split_timers]))
+                     for k in ops.STAGES}
+        flat = ids.reshape(-1).long()
+        counts = torch.bincount(flat[flat >= 0], minlength=cfg.E)  # padding tokens have ids -1
+        experts_used = int((counts > 0).sum().item())
 
     # end to end: pinned host tokens -> device -> block -> host, every step.
     # Serial: one batch at a time, the copies on the compute stream.
@@ -349,7 +388,7 @@ def run_ours(args, world, rank, local):
     _barrier(world)
     e2e_serial_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     e2e_ms, e2e_mode = e2e_serial_ms, "serial: copy in, block, copy out, one batch at a time"
-    if layers == 1 and mask_dev is None:
+    if layers == 1 and mask_dev is None and not dense:
         # the library's host-batch entry point: every step's batch is copied in
         # and its output copied out, the copies of the neighbouring batches
         # overlapping each batch's kernels (two copy streams)
@@ -381,7 +420,7 @@ def run_ours(args, world, rank, local):
         tok_per_step = wl.T * layers
         total_tokens = tok_per_step * world
         value = total_tokens / (ms * 1e-3)
-        fpt = flops_per_token(cfg)
+        fpt = flops_per_token(cfg) if not dense else 6.0 * wl.H * wl.dense_I
         # padding tokens (token mask 0) run only the router and the shared expert
         n_pad = 0 if mask_dev is None else int((mask_dev == 0).sum().item())
         n_real = wl.T - n_pad
@@ -393,6 +432,8 @@ def run_ours(args, world, rank, local):
         R = n_real * cfg.top_k
         up_rows = R + (wl.T if cfg.I_shared == cfg.I else 0)
         up_flops = 2.0 * up_rows * cfg.H * (2 * cfg.I)
+        if dense:  # the timed launch pair is the whole layer: both GEMMs
+            up_rows, up_flops = wl.T, flops_per_step
         up_ms = up_ms_live
         # a kernel inside a long timed region runs at the power-capped sustained
         # clock: compare it with the sustained peak there, with the burst peak otherwise
@@ -401,13 +442,17 @@ def run_ours(args, world, rank, local):
         peak_tf = peaks.get(peak_key, peaks["bf16_tflops"])
         achieved = up_flops / (up_ms * 1e-3) / 1e12
         layer_ms = ms / layers
-        hbm_bytes = algorithmic_bytes(cfg, experts_used)
+        hbm_bytes = (algorithmic_bytes(cfg, experts_used) if not dense else
+                     3.0 * wl.dense_I * wl.H * 2 + 2.0 * wl.T * wl.H * 2)
         t_flop = flops_per_step / peak_tf / 1e12
         t_hbm = hbm_bytes / peaks["hbm_gbs"] / 1e9
         swapped = wl.T * cfg.top_k <= 64 * cfg.E  # the kernel the library picks for this shape
         kernel = ("grouped_gemm_swap_kernel<SwiGLU> (expert up, shared expert folded in)"
                   if swapped else
                   "grouped_gemm_kernel<SwiGLU> (expert up, shared expert folded in)")
+        if dense:
+            swapped = wl.T <= 64
+            kernel = "grouped_gemm_kernel<SwiGLU> + <RowScale> (dense layer: both GEMMs)"
         if t_hbm > t_flop:
             # HBM-bound layer: the expert-up launch streams w13 of the used experts and
             # ws13, reads the gathered rows and x, writes h
@@ -423,7 +468,7 @@ def run_ours(args, world, rank, local):
                   "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                   "frac": achieved / peak_tf,
                   "peak_source": f"{peak_src} bf16 dense {'sustained' if long_region else 'burst'}"}
-        rf["traffic"] = (None if swapped else
+        rf["traffic"] = (None if swapped or dense else
                          measured_traffic("grouped_gemm_kernel<EPI_SWIGLU>", wl.name))
         rf["traffic_unit"] = "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
         rf["layer_roofline_frac"] = max(t_flop, t_hbm) / (layer_ms * 1e-3)
@@ -440,11 +485,15 @@ def run_ours(args, world, rank, local):
                        "topk_group": cfg.topk_group, "layers": layers,
                        "tokens_per_gpu_per_step": tok_per_step,
                        "padding_tokens_per_layer": n_pad,
-                       "l2": "inputs larger than L2: 1.2 GB of expert weights read per layer"},
+                       "dense_intermediate": wl.dense_I or None,
+                       "l2": ("inputs larger than L2: " +
+                              ("the layer's 85 MB of weights, 80 MB of tokens in and out"
+                               if dense else "1.2 GB of expert weights read per layer"))},
             "tflops": tflops,
             "roofline": rf,
             "stage_ms": per_stage,
-            "stage_ms_note": "separate pass with an event at every stage boundary",
+            "stage_ms_note": ("the timed calls themselves" if dense else
+                              "separate pass with an event at every stage boundary"),
             "experts_used": experts_used,
             "cpu_baseline": None if cpu_tps is None else {
                 "value": cpu_tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -454,7 +503,8 @@ def run_ours(args, world, rank, local):
                     "d2h_bytes_per_step": int(out_host.numel() * 2),
                     "mode": e2e_mode,
                     "serial_value": total_tokens / (e2e_serial_ms * 1e-3)},
-            "gpu_launches": (KERNELS_PER_STEP + (1 if layers > 1 else 0)) * layers * args.steps,
+            "gpu_launches": ((2 if dense else KERNELS_PER_STEP + (1 if layers > 1 else 0)) *
+                             layers * args.steps),
             "clocks": sampler.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -247,6 +247,25 @@ MOE_API int32_t moe_forward_host(const void* const* x_host, void* const* out_hos
                                  size_t workspace_bytes, void* stream, void* h2d_stream,
                                  void* d2h_stream);
 
+/* Dense feed-forward layer ([S2] "MoE 实现的源码级要点": a transformer block
+ * uses the sparse MoE block or a plain LingBotVideoMLP -- the dense FFN -- by
+ * decoder_sparse_step and layer index; the shared expert is the same MLP):
+ *   out = bf16( [residual +] SwiGLU(x) ),  SwiGLU(x) = (silu(x.Wg^T) * (x.Wu^T)) . W2^T
+ *   x        device bf16 [T,H]
+ *   w13      device bf16 [2I,H]   gate rows 0..I-1, up rows I..2I-1 (non-interleaved)
+ *   w2       device bf16 [H,I]
+ *   residual device bf16 [T,H] or NULL; may be the same buffer as out
+ *   out      device bf16 [T,H], must not overlap x
+ *   workspace device, moe_dense_ffn_workspace_bytes(T,H,I) bytes, 256-byte aligned
+ * H and I multiples of 64 (<= 16384).  The intermediate h is stored in bf16;
+ * with a residual the MLP output is stored in bf16 and added to the residual
+ * in fp32 with one final rounding (as the block's restore).  Device-side
+ * errors go to the workspace status word (moe_read_device_status). */
+MOE_API size_t moe_dense_ffn_workspace_bytes(int32_t T, int32_t H, int32_t I);
+MOE_API int32_t moe_dense_ffn(const void* x, const void* w13, const void* w2, int32_t T,
+                              int32_t H, int32_t I, const void* residual, void* out,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
 /* RMSNorm with fp32 accumulation ([S2]: RMSNorm accumulates in fp32), for a
  * residual stack of blocks: xn = bf16(x * rsqrt(mean(x^2) + eps) * gamma).
  *   x device bf16 [T,H]; gamma device fp32 [H] or NULL (= 1); xn device bf16 [T,H]. */

@@ -20,6 +20,8 @@ from .moe_oracle import (  # noqa: F401
     route,
     routing_weights,
     swiglu_mlp,
+    dense_ffn,
+    apply_token_mask,
     moe_forward,
     moe_forward_tokens,
     permutation,

@@ -238,6 +238,18 @@ def swiglu_mlp(x: np.ndarray, w13: np.ndarray, w2: np.ndarray) -> np.ndarray:
     return (_silu(gate) * up) @ w2.astype(np.float64).T
 
 
+def dense_ffn(x: np.ndarray, w13: np.ndarray, w2: np.ndarray, residual=None) -> np.ndarray:
+    """Dense feed-forward layer ([S2] "MoE 实现的源码级要点": a block uses the sparse
+    MoE block or a plain LingBotVideoMLP -- the dense FFN -- by decoder_sparse_step
+    and layer index; the shared expert is the same MLP).  float64 [T,H]:
+    out = SwiGLU(x; w13 [2I,H] gate|up, w2 [H,I]) (+ residual).  Pinned through
+    ``swiglu_mlp``'s pins."""
+    out = swiglu_mlp(x, w13, w2)
+    if residual is not None:
+        out = out + residual.astype(np.float64)
+    return out
+
+
 def moe_forward(x, Wr, bias, w13, w2, ws13, ws2, cfg: MoeConfig,
                 residual=None, ids=None, token_mask=None):
     """Block output in float64 [T,H].

@@ -615,6 +615,82 @@ int32_t moe_forward_host(const void* const* x_host, void* const* out_host, int32
   return MOE_OK;
 }
 
+size_t moe_dense_ffn_workspace_bytes(int32_t T, int32_t H, int32_t I) {
+  if (T < 0 || H <= 0 || I <= 0 || H % 64 != 0 || I % 64 != 0 || H > MAX_DIM || I > MAX_DIM)
+    return 0;
+  // status, h [T,I], the MLP output [T,H] (added to a residual)
+  return align_up(sizeof(DevStatus)) + align_up((size_t)T * I * 2) + align_up((size_t)T * H * 2);
+}
+
+int32_t moe_dense_ffn(const void* x, const void* w13, const void* w2, int32_t T, int32_t H,
+                      int32_t I, const void* residual, void* out, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (T < 0 || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+  if (H % 64 != 0 || I % 64 != 0 || H > MAX_DIM || I > MAX_DIM) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!x || !w13 || !w2 || !out || out == x) return MOE_ERR_INVALID_ARG;
+  if (!ws_ok(workspace, workspace_bytes, moe_dense_ffn_workspace_bytes(T, H, I)))
+    return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = at<int>(workspace, 0);
+  __nv_bfloat16* h = at<__nv_bfloat16>(workspace, align_up(sizeof(DevStatus)));
+  __nv_bfloat16* y =
+      at<__nv_bfloat16>(workspace, align_up(sizeof(DevStatus)) + align_up((size_t)T * I * 2));
+  __nv_bfloat16* dst = residual ? y : static_cast<__nv_bfloat16*>(out);
+  RMOE_TRY(launch_status_reset(status, s));
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.status = status;
+  a.timeout_ns = DEFAULT_TIMEOUT_NS;
+  a.alt_group = -1;
+  a.single_rows = T;  // one group: every row uses the same weights
+  const int sms = num_sms();
+  GemmArgs up = a, down = a;
+  up.k_steps = H / 64;
+  up.b_second = I;
+  up.out = h;
+  up.ldo = I;
+  up.n_valid = I;
+  down.k_steps = I / 64;
+  down.out = dst;
+  down.ldo = H;
+  down.n_valid = H;
+  down.dest_mul = 1;  // output row = row
+  if (T <= 64) {  // few rows: the swapped GEMMs, which stream the weights once
+    const int chunk = T <= 20 ? 32 : 128;
+    CUtensorMap tm_w13, tm_x, tm_w2, tm_h;
+    RMOE_TRY(make_tmap_3d(&tm_w13, w13, 1, 2 * (uint64_t)I, H));
+    RMOE_TRY(make_tmap_2d_box(&tm_x, x, T, H, 32));
+    RMOE_TRY(make_tmap_3d(&tm_w2, w2, 1, H, I));
+    RMOE_TRY(make_tmap_2d_box(&tm_h, h, T, I, 32));
+    up.n_tiles = (I + 127) / 128;
+    up.n_out_tile = 128;
+    down.n_tiles = (H + 127) / 128;
+    down.n_out_tile = 128;
+    RMOE_TRY(launch_grouped_gemm_swap(EPI_SWIGLU, chunk, tm_w13, tm_x, tm_w13, tm_x, up, sms, s));
+    RMOE_TRY(launch_grouped_gemm_swap(EPI_ROWSCALE, chunk, tm_w2, tm_h, tm_w2, tm_h, down, sms, s));
+  } else {
+    CUtensorMap tm_w13, tm_x, tm_w2, tm_h;
+    RMOE_TRY(make_tmap_3d(&tm_w13, w13, 1, 2 * (uint64_t)I, H));
+    RMOE_TRY(make_tmap_2d(&tm_x, x, T, H));
+    RMOE_TRY(make_tmap_3d(&tm_w2, w2, 1, H, I));
+    RMOE_TRY(make_tmap_2d(&tm_h, h, T, I));
+    const int mt = (T + MTILE - 1) / MTILE;
+    up.n_tiles = (I + 127) / 128;
+    up.n_out_tile = 128;
+    down.n_tiles = (H + 255) / 256;
+    down.n_out_tile = 256;
+    down.b_second = 128;
+    RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_x, tm_w13, tm_x, tm_w13, up,
+                                 std::min(sms, 2 * mt * up.n_tiles), s));
+    RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, tm_h, tm_w2, down,
+                                 std::min(sms, 2 * mt * down.n_tiles), s));
+  }
+  if (residual)  // out = bf16(residual + y), fp32 sum, one rounding
+    RMOE_TRY(launch_combine_slots(y, nullptr, 0, T, H, 1, residual, out, s));
+  return MOE_OK;
+}
+
 int32_t moe_rmsnorm(const void* x, const float* gamma, float eps, int32_t T, int32_t H, void* xn,
                     void* stream) {
   if (T < 0 || H <= 0 || H % 64 != 0 || H > MAX_DIM || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;

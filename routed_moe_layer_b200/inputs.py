@@ -32,6 +32,8 @@ import torch
 #   4: 48 residual layers x (RMSNorm -> block) at 19412 tokens, H=2048
 #   5: CFG batch 2 x 19412 rows with padded text: the second prompt has 64 real
 #      text tokens, its other 448 text rows are padding (token mask 0)
+#   6: dense feed-forward layer (a block without experts), 19412 tokens, H=2048,
+#      intermediate 6912 = 9 x 768 (the active width of one token of the MoE block)
 HOT_EXPERTS = tuple(range(0, 128, 16))  # two per group of 32
 
 
@@ -45,6 +47,7 @@ class Workload:
     hot_experts: Optional[Sequence[int]] = None
     hot_bias: float = 0.5
     padding: Optional[Sequence[tuple]] = None  # [start, stop) row ranges of padding tokens
+    dense_I: int = 0  # > 0: a dense feed-forward layer of this intermediate size
 
 
 WORKLOADS = {
@@ -55,6 +58,7 @@ WORKLOADS = {
     4: Workload("moe_stack48_T19412_H2048", 19412, 2048, 4, layers=48),
     5: Workload("moe_layer_cfg2x19412_H2048_padded", 38824, 2048, 5,
                 padding=((19412 + 18900 + 64, 38824),)),
+    6: Workload("dense_ffn_T19412_H2048_I6912", 19412, 2048, 6, dense_I=6912),
 }
 
 
@@ -109,6 +113,14 @@ def make_weights(H: int, seed: int, E: int = 128, I: int = 768, I_shared: int = 
     return dict(Wr=Wr, bias=bias, w13=w13, w2=w2, ws13=ws13, ws2=ws2)
 
 
+def make_dense_weights(H: int, I: int, seed: int, device="cpu", std: float = 0.02):
+    """Returns dict(w13 [2I,H], w2 [H,I]) of a dense feed-forward layer
+    (tensor indices 3 and 4 of the recipe)."""
+    base = seed * 1000
+    return dict(w13=_normal((2 * I, H), std, base + 3, device, torch.bfloat16),
+                w2=_normal((H, I), std, base + 4, device, torch.bfloat16))
+
+
 def make_block_inputs(T: int, H: int, seed: int, E: int = 128, I: int = 768,
                       I_shared: int = 768, device="cpu", hot_experts=None,
                       hot_bias: float = 0.5, unit_scale: bool = False):
@@ -128,7 +140,10 @@ def make_block_inputs(T: int, H: int, seed: int, E: int = 128, I: int = 768,
 def workload_inputs(cfg_id: int, device="cpu", layer: int = 0):
     """Inputs of a named workload (for a stack: the tokens and layer ``layer``)."""
     w = WORKLOADS[cfg_id]
-    d = make_weights(w.H, w.seed, device=device, layer=layer,
-                     hot_experts=w.hot_experts, hot_bias=w.hot_bias)
+    if w.dense_I:
+        d = make_dense_weights(w.H, w.dense_I, w.seed, device=device)
+    else:
+        d = make_weights(w.H, w.seed, device=device, layer=layer,
+                         hot_experts=w.hot_experts, hot_bias=w.hot_bias)
     d["x"] = make_tokens(w.T, w.H, w.seed, device=device)
     return d

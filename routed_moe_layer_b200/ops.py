@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
         "moe_forward_host_workspace_bytes": (sz, [cfgp]),
         "moe_forward_host": (i32, [ctypes.POINTER(vp), ctypes.POINTER(vp), i32, vp, vp, vp, vp,
                                    vp, vp, cfgp, vp, sz, vp, vp, vp]),
+        "moe_dense_ffn_workspace_bytes": (sz, [i32, i32, i32]),
+        "moe_dense_ffn": (i32, [vp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
         "moe_rmsnorm": (i32, [vp, vp, ctypes.c_float, i32, i32, vp, vp]),
         "moe_read_device_status": (i32, [vp, ctypes.POINTER(i32), vp]),
         "moe_selftest_wait_timeout": (i32, [vp, i64, vp]),
@@ -340,6 +342,28 @@ def forward_host(x_host: Sequence[torch.Tensor], out_host: Sequence[torch.Tensor
                                   workspace.numel(), _stream_ptr(), h2d, d2h),
            "moe_forward_host")
     return workspace
+
+
+def dense_ffn(x: torch.Tensor, w13: torch.Tensor, w2: torch.Tensor,
+              residual: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+              workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Dense SwiGLU feed-forward layer (moe_dense_ffn): out = [residual +] SwiGLU(x)."""
+    T, H = x.shape
+    I = w13.shape[0] // 2
+    _need(x, "x", torch.bfloat16, (T, H))
+    _need(w13, "w13", torch.bfloat16, (2 * I, H))
+    _need(w2, "w2", torch.bfloat16, (H, I))
+    if residual is not None:
+        _need(residual, "residual", torch.bfloat16, (T, H))
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    else:
+        _need(out, "out", torch.bfloat16, (T, H))
+    if workspace is None:
+        workspace = alloc_workspace(lib().moe_dense_ffn_workspace_bytes(T, H, I), x.device)
+    _check(lib().moe_dense_ffn(_ptr(x), _ptr(w13), _ptr(w2), T, H, I, _ptr(residual), _ptr(out),
+                               _ptr(workspace), workspace.numel(), _stream_ptr()), "moe_dense_ffn")
+    return out
 
 
 def rmsnorm(x: torch.Tensor, gamma: Optional[torch.Tensor] = None, eps: float = 1e-6,

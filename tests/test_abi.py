@@ -171,3 +171,21 @@ def test_forward_host_rejects_bad_arguments_on_the_host(L):
     assert call(None, None, 0) == 0
     z = BlockConfig(T=0, H=256, I=128, I_shared=128).c()
     assert call(None, None, 3, cfg=z) == 0
+
+
+def test_dense_ffn_rejects_bad_arguments_on_the_host(L):
+    need = L.moe_dense_ffn_workspace_bytes(64, 256, 128)
+    assert need >= 64 * 128 * 2 + 64 * 256 * 2
+    assert L.moe_dense_ffn_workspace_bytes(64, 250, 128) == 0
+    out = ctypes.c_void_p(0x20000)
+    args = lambda **k: [k.get("x", FAKE), FAKE, FAKE, k.get("T", 64), k.get("H", 256),
+                        k.get("I", 128), None, k.get("out", out), k.get("ws", FAKE),
+                        k.get("nbytes", need), None]
+    assert L.moe_dense_ffn(*args(x=None)) == 1
+    assert L.moe_dense_ffn(*args(out=FAKE)) == 1          # out aliases x
+    assert L.moe_dense_ffn(*args(T=-1)) == 1
+    assert L.moe_dense_ffn(*args(H=250)) == 2
+    assert L.moe_dense_ffn(*args(I=16384 + 64)) == 2
+    assert L.moe_dense_ffn(*args(nbytes=need - 1)) == 3
+    assert L.moe_dense_ffn(*args(ws=ctypes.c_void_p(0x10010))) == 3
+    assert L.moe_dense_ffn(*args(T=0, x=None, out=None)) == 0

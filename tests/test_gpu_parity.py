@@ -353,6 +353,32 @@ def test_forward_host_batches_match_device_forward(overlap):
     parity.check_output(outs[1], ids_b, d_np, cfg)
 
 
+@pytest.mark.parametrize("T,H,I", [(1, 256, 128), (40, 512, 192), (64, 320, 256),
+                                   (300, 512, 256), (1000, 1024, 768), (2048, 2048, 1536)])
+def test_dense_ffn_matches_oracle(T, H, I):
+    """Dense feed-forward layer (up to 64 rows: swapped GEMMs, else tiled), with
+    and without a residual (also in place)."""
+    g = torch.Generator().manual_seed(T + I)
+    x = torch.randn((T, H), generator=g).to(torch.bfloat16)
+    w13 = (torch.randn((2 * I, H), generator=g) * H ** -0.5).to(torch.bfloat16)
+    w2 = (torch.randn((H, I), generator=g) * I ** -0.5).to(torch.bfloat16)
+    res = torch.randn((T, H), generator=g).to(torch.bfloat16)
+    xd, w13d, w2d, resd = (t.to(DEV) for t in (x, w13, w2, res))
+    out = ops.dense_ffn(xd, w13d, w2d)
+    out_r = ops.dense_ffn(xd, w13d, w2d, residual=resd)
+    buf = resd.clone()
+    ops.dense_ffn(xd, w13d, w2d, residual=buf, out=buf)
+    torch.cuda.synchronize()
+    assert torch.equal(buf, out_r)
+    xn, w13n, w2n, resn = (parity.to_np(t) for t in (x, w13, w2, res))
+    for got, ref in ((out, oracle.dense_ffn(xn, w13n, w2n)),
+                     (out_r, oracle.dense_ffn(xn, w13n, w2n, residual=resn))):
+        g_np = parity.to_np(got).astype(np.float64)
+        err = np.abs(g_np - ref)
+        assert np.all(err <= parity.OUT_RTOL * (1 + np.abs(ref))), err.max()
+        assert np.sqrt(np.mean(err ** 2) / np.mean(ref ** 2)) < 1e-2
+
+
 # ------------------------------------------------------------------ RMSNorm, residual stack
 def test_rmsnorm_matches_oracle():
     T, H = 333, 2048
