@@ -57,20 +57,24 @@ __global__ void __launch_bounds__(256)
 // in fp32 in slot order, then adds the residual, then rounds once.
 __global__ void __launch_bounds__(256)
     combine_slots_kernel(const __nv_bfloat16* __restrict__ Y, const int* __restrict__ row_of,
-                         int top_k, int T, int H, int slots,
+                         int top_k, int T, int H, int slots, int parts,
                          const __nv_bfloat16* __restrict__ residual,
                          __nv_bfloat16* __restrict__ out) {
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (blockDim.x >> 5);
-  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+  // `parts` warps share a token (small batches), each taking every parts-th
+  // 512-byte column block of the row
+  for (int wt = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); wt < T * parts;
+       wt += warps) {
+    const int t = wt / parts, part = wt - t * parts;
     uint32_t skip = 0;  // routed slots of rejected expert ids
     for (int j = 0; j < top_k; ++j)
       if (row_of[(size_t)t * top_k + j] < 0) skip |= 1u << j;
     const uint4* src = reinterpret_cast<const uint4*>(Y + (size_t)t * slots * H);
     const int hv = H / 8;  // 16-byte vectors per row
-    for (int c = lane; c < hv; c += 32) {
+    for (int c = lane + 32 * part; c < hv; c += 32 * parts) {
       float s[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) s[i] = 0.f;
@@ -132,11 +136,17 @@ cudaError_t launch_rmsnorm(const void* x, const float* gamma, float eps, int T, 
 
 cudaError_t launch_combine_slots(const void* Y, const int* row_of, int top_k, int T, int H,
                                  int slots, const void* residual, void* out, cudaStream_t stream) {
-  int grid = (T + 7) / 8;
-  const int cap = num_sms() * 8;
+  // warps per token: enough warps to fill the GPU twice over, at most one per
+  // 512-byte column block of a row
+  const int cap = num_sms() * 8;  // blocks of 8 warps
+  int parts = (2 * cap * 8) / (T > 0 ? T : 1);
+  const int max_parts = H / 256;
+  if (parts > max_parts) parts = max_parts;
+  if (parts < 1) parts = 1;
+  long long grid = ((long long)T * parts + 7) / 8;
   if (grid > cap) grid = cap;
-  return launch_chained(combine_slots_kernel, dim3(grid), dim3(256), 0, stream,
-                        static_cast<const __nv_bfloat16*>(Y), row_of, top_k, T, H, slots,
+  return launch_chained(combine_slots_kernel, dim3((unsigned)grid), dim3(256), 0, stream,
+                        static_cast<const __nv_bfloat16*>(Y), row_of, top_k, T, H, slots, parts,
                         static_cast<const __nv_bfloat16*>(residual),
                         static_cast<__nv_bfloat16*>(out));
 }

@@ -190,10 +190,13 @@ __global__ void __launch_bounds__(1024)
   const int t = tid;
   const bool real = t < T && (!tmask || tmask[t] != 0);  // padding tokens take no rows
   int my_e[MAX_TOPK_PERMUTE];
+  float my_w[MAX_TOPK_PERMUTE];  // loaded with the ids, off the scatter's critical path
 #pragma unroll
   for (int j = 0; j < MAX_TOPK_PERMUTE; ++j) {
     my_e[j] = -1;
+    my_w[j] = 1.0f;
     if (real && j < top_k) {
+      if (topk_w) my_w[j] = topk_w[(size_t)t * top_k + j];
       const int e = ids[(size_t)t * top_k + j];
       if (e >= 0 && e < E) {
         my_e[j] = e;
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(1024)
     const int row = excl_rows[e] + wbase[warp][e] + __popc(masks[warp][e] & lower);
     row_of[tj] = row;
     tok_of[row] = t;
-    if (w_of) w_of[row] = topk_w ? topk_w[tj] : 1.0f;
+    if (w_of) w_of[row] = my_w[j];
     if (pos_of) pos_of[row] = t * slot_stride + j;
   }
 }
@@ -275,23 +278,30 @@ __global__ void __launch_bounds__(PT)
   }
 }
 
-// One warp per token: x[t] is read once (512 bytes per warp step) and written
-// to the token's top_k rows; row_of gives them (-1: skipped id).
+// One warp per token: x[t] is read once (1 KB per warp step: 32 bytes per
+// lane) and written to the token's top_k rows with full-sector stores;
+// row_of gives the rows (-1: skipped id), fetched once per token.
 __global__ void __launch_bounds__(256)
     gather_tokens_kernel(const __nv_bfloat16* __restrict__ x, const int* __restrict__ row_of,
                          int T, int H, int top_k, __nv_bfloat16* __restrict__ xp) {
+  __shared__ int rows_sm[8][MAX_TOPK_PERMUTE];  // each warp's current token's rows
   pdl_launch_dependents();
   pdl_wait();
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int warps = gridDim.x * (blockDim.x >> 5);
-  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
-    const int my_row = lane < top_k ? row_of[(size_t)t * top_k + lane] : -1;
+  const int chunks = H / 16;  // 32-byte pieces of a row (H is a multiple of 64)
+  int* rows = rows_sm[wib];
+  for (int t = blockIdx.x * (blockDim.x >> 5) + wib; t < T; t += warps) {
+    __syncwarp();  // the previous token's rows have been used
+    if (lane < top_k) rows[lane] = row_of[(size_t)t * top_k + lane];
+    __syncwarp();
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
-    for (int c = lane; c < H / 8; c += 32) {
-      const uint4 v = src[c];
+    for (int c = lane; c < chunks; c += 32) {
+      const uint4 a = src[2 * c], b = src[2 * c + 1];
+      const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
       for (int j = 0; j < top_k; ++j) {
-        const int r = __shfl_sync(0xffffffffu, my_row, j);
-        if (r >= 0) reinterpret_cast<uint4*>(xp + (size_t)r * H)[c] = v;
+        const int r = rows[j];
+        if (r >= 0) st_global_v8(xp + (size_t)r * H + 16 * c, v);
       }
     }
   }
