@@ -438,11 +438,16 @@ cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint
 
 cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, uint64_t groups, uint64_t n_rows,
                          uint64_t K) {
+  return make_tmap_3d_box(map, base, groups, n_rows, K, BN / 2);
+}
+
+cudaError_t make_tmap_3d_box(CUtensorMap* map, const void* base, uint64_t groups,
+                             uint64_t n_rows, uint64_t K, uint32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   const cuuint64_t dims[3] = {K, n_rows, groups};
   const cuuint64_t strides[2] = {K * 2, n_rows * K * 2};
-  const cuuint32_t box[3] = {BK, BN / 2, 1};
+  const cuuint32_t box[3] = {BK, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,

@@ -103,6 +103,9 @@ cudaError_t make_tmap_2d_box(CUtensorMap* map, const void* base, uint64_t rows, 
                              uint32_t box_rows);
 cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, uint64_t groups, uint64_t n_rows,
                          uint64_t K);
+// The same with a box of box_rows rows.
+cudaError_t make_tmap_3d_box(CUtensorMap* map, const void* base, uint64_t groups,
+                             uint64_t n_rows, uint64_t K, uint32_t box_rows);
 
 // tmA2/tmB2 serve group args.alt_group (A rows re-based to 0, B group 0).
 cudaError_t launch_grouped_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,

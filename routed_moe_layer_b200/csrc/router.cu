@@ -40,7 +40,7 @@ constexpr int R_B_BYTES = RBN * RBK * 2;
 constexpr int R_STAGE_BYTES = R_A_BYTES + 3 * R_B_BYTES;
 constexpr int R_THREADS = 192;
 constexpr uint32_t R_TMEM_COLS = 256;  // two 128-column accumulators
-constexpr uint32_t R_IDESC = idesc_bf16_f32(RBM, RBN);
+constexpr int R_NP_SMALL = 32;  // expert columns per item when the batch is small
 
 struct __align__(8) RouterTail {
   uint64_t full[RSTAGES];
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(R_THREADS, 1)
     router_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmW3, int T, int E, int k_steps,
-                       int S, float* __restrict__ partial, int* status,
+                       int S, int NP, float* __restrict__ partial, int* status,
                        unsigned long long timeout_ns) {
   pdl_launch_dependents();
   pdl_wait();
@@ -100,7 +100,12 @@ __global__ void __launch_bounds__(R_THREADS, 1)
                                              ~static_cast<uintptr_t>(1023));
   RouterTail& st = *reinterpret_cast<RouterTail*>(smem + (size_t)RSTAGES * R_STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int items = ((T + RBM - 1) / RBM) * S;
+  // item = (token tile, K chunk, part of NP expert columns); NP < 128 gives
+  // small batches more CTAs without changing any logit's arithmetic
+  const int parts = (RBN + NP - 1) / NP;
+  const int items = ((T + RBM - 1) / RBM) * S * parts;
+  const uint32_t idesc = idesc_bf16_f32(RBM, NP);
+  const uint32_t b_bytes = (uint32_t)NP * RBK * 2;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < RSTAGES; ++i) {
@@ -137,7 +142,8 @@ __global__ void __launch_bounds__(R_THREADS, 1)
       uint32_t armed = 0, armed_parity = 0;
       bool ok = true;
       for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
-        const int m0 = (it / S) * RBM, s = it % S;
+        const int ms = it / parts, n0 = (it - ms * parts) * NP;
+        const int m0 = (ms / S) * RBM, s = ms % S;
         const int kb = (int)((long long)s * k_steps / S);
         const int ke = (int)((long long)(s + 1) * k_steps / S);
         for (int k = kb; k < ke; ++k) {
@@ -146,11 +152,11 @@ __global__ void __launch_bounds__(R_THREADS, 1)
             break;
           }
           uint8_t* sa = smem + (size_t)stage * R_STAGE_BYTES;
-          mbar_arrive_expect_tx(&st.full[stage], R_STAGE_BYTES);
+          mbar_arrive_expect_tx(&st.full[stage], R_A_BYTES + 3 * b_bytes);
           tma_load_2d(sa, &tmX, &st.full[stage], k * RBK, m0);
 #pragma unroll
           for (int t = 0; t < 3; ++t)
-            tma_load_3d(sa + R_A_BYTES + t * R_B_BYTES, &tmW3, &st.full[stage], k * RBK, 0, t);
+            tma_load_3d(sa + R_A_BYTES + t * R_B_BYTES, &tmW3, &st.full[stage], k * RBK, n0, t);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == RSTAGES) {
@@ -173,7 +179,7 @@ __global__ void __launch_bounds__(R_THREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
-        const int s = it % S;
+        const int s = (it / parts) % S;
         const int kb = (int)((long long)s * k_steps / S);
         const int ke = (int)((long long)(s + 1) * k_steps / S);
         if (!mbar_wait(&st.tempty[acc], acc_phase ^ 1u, wc, 43)) break;
@@ -192,7 +198,7 @@ __global__ void __launch_bounds__(R_THREADS, 1)
             const uint64_t db = sdesc_kmajor_sw128(sa + R_A_BYTES + t * R_B_BYTES);
 #pragma unroll
             for (int kk = 0; kk < RBK / 16; ++kk)
-              umma_bf16_ss(d_tmem, da + 2 * kk, db + 2 * kk, R_IDESC,
+              umma_bf16_ss(d_tmem, da + 2 * kk, db + 2 * kk, idesc,
                            (k != kb || t != 0 || kk != 0) ? 1u : 0u);
           }
           umma_commit(&st.empty[stage]);
@@ -215,27 +221,28 @@ __global__ void __launch_bounds__(R_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x) {
-      const int m0 = (it / S) * RBM, s = it % S;
+      const int ms = it / parts, n0 = (it - ms * parts) * NP;
+      const int m0 = (ms / S) * RBM, s = ms % S;
       const bool ok = mbar_wait(&st.tfull[acc], acc_phase, wc, 42);
       if (!__all_sync(FULL, ok)) break;
       tc_fence_after_sync();
       const int row = m0 + q * 32 + lane;
-      float* dst = partial + ((size_t)s * T + row) * E;
+      float* dst = partial + ((size_t)s * T + row) * E + n0;
       const uint32_t tbase =
           tmem_base + static_cast<uint32_t>(acc * RBN) + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < RBN; c += 32) {
+      for (int c = 0; c < NP; c += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + c, v);
         tmem_ld_wait();
-        if (row < T && c < E) {
-          if (c + 32 <= E && (E & 7) == 0) {
+        if (row < T && n0 + c < E) {
+          if (n0 + c + 32 <= E && (E & 7) == 0) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) st_global_v8(dst + c + 8 * i, v + 8 * i);
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              if (c + i < E) dst[c + i] = __uint_as_float(v[i]);
+              if (n0 + c + i < E) dst[c + i] = __uint_as_float(v[i]);
           }
         }
       }
@@ -420,19 +427,22 @@ cudaError_t launch_router(const void* x, const float* Wr, const float* bias, con
   cudaError_t err = launch_chained(router_split_kernel, dim3(split_grid), dim3(256), 0, stream, Wr,
                                    n, Wr3, status, p.clear_status);
   if (err != cudaSuccess) return err;
+  const int S = router_splits(H);
+  // split the expert columns when token tiles x K chunks leave most SMs idle
+  const int tiles = ((T + RBM - 1) / RBM) * S;
+  const int NP = tiles * (RBN / R_NP_SMALL) <= num_sms() ? R_NP_SMALL : RBN;
   CUtensorMap tmX, tmW3;
   err = make_tmap_2d(&tmX, x, (uint64_t)T, (uint64_t)H);
   if (err != cudaSuccess) return err;
-  err = make_tmap_3d(&tmW3, Wr3, 3, (uint64_t)E, (uint64_t)H);
+  err = make_tmap_3d_box(&tmW3, Wr3, 3, (uint64_t)E, (uint64_t)H, (uint32_t)NP);
   if (err != cudaSuccess) return err;
   err = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)R_SMEM_BYTES);
   if (err != cudaSuccess) return err;
-  const int S = router_splits(H);
-  const int items = ((T + RBM - 1) / RBM) * S;
+  const int items = tiles * (RBN / NP);
   const int grid = items < num_sms() ? items : num_sms();
   err = launch_chained(router_gemm_kernel, dim3(grid), dim3(R_THREADS), R_SMEM_BYTES, stream, tmX,
-                       tmW3, T, E, H / RBK, S, partial, status, timeout_ns);
+                       tmW3, T, E, H / RBK, S, NP, partial, status, timeout_ns);
   if (err != cudaSuccess) return err;
   int sel_grid = ((T + 1) / 2 + SEL_WARPS - 1) / SEL_WARPS;
   const int cap = num_sms() * 16;
