@@ -41,6 +41,7 @@ constexpr int R_STAGE_BYTES = R_A_BYTES + 3 * R_B_BYTES;
 constexpr int R_THREADS = 192;
 constexpr uint32_t R_TMEM_COLS = 256;  // two 128-column accumulators
 constexpr int R_NP_SMALL = 32;  // expert columns per item when the batch is small
+constexpr int ROUTER_WARP_SELECT_MAX_T = 4096;  // one warp per token up to this many tokens
 
 struct __align__(8) RouterTail {
   uint64_t full[RSTAGES];
@@ -403,6 +404,147 @@ __global__ void __launch_bounds__(SEL_WARPS * 32)
   }
 }
 
+// One warp per token: lane l holds experts l + 32*i (i < 4).  The same
+// arithmetic as router_select_kernel (logit sum order, sigmoid, c = s + bias,
+// group score = the two largest c summed, ranking and tie rules, weights
+// summed in selection order), with shorter dependency chains: every group's
+// top-2 is merged across the warp by shuffles, and each selection round is one
+// 4-slot scan plus a 5-level argmax.  Used for small batches (latency-bound).
+__device__ __forceinline__ void warp_argmax(float& v, int& idx) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ov = __shfl_xor_sync(FULL, v, off);
+    const int oi = __shfl_xor_sync(FULL, idx, off);
+    if (ov > v || (ov == v && oi < idx)) {
+      v = ov;
+      idx = oi;
+    }
+  }
+}
+
+constexpr int W1_NE = RBN / 32;  // expert slots per lane
+
+__global__ void __launch_bounds__(256)
+    router_select_warp_kernel(const float* __restrict__ partial, int S,
+                              const float* __restrict__ bias, RouterParams p,
+                              int32_t* __restrict__ topk_ids, float* __restrict__ topk_w) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int T = p.T, E = p.E;
+  const int gs = E / p.n_group;
+  const bool group_step = p.topk_group < p.n_group;
+  float b[W1_NE];
+  int gid[W1_NE];
+#pragma unroll
+  for (int i = 0; i < W1_NE; ++i) {
+    const int e = lane + 32 * i;
+    b[i] = e < E ? bias[e] : 0.f;
+    gid[i] = e < E ? e / gs : -1;
+  }
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+    float s[W1_NE], c[W1_NE];
+    uint32_t avail = 0;
+#pragma unroll
+    for (int i = 0; i < W1_NE; ++i) {
+      const int e = lane + 32 * i;
+      s[i] = 0.f;
+      c[i] = -FLT_MAX;
+      if (e < E) {
+        float l = partial[(size_t)t * E + e];
+        for (int k = 1; k < S; ++k) l += partial[((size_t)k * T + t) * E + e];
+        s[i] = __frcp_rn(1.0f + expf(-l));  // correctly rounded: the same value as 1/(1+e^-l)
+        c[i] = s[i] + b[i];
+        avail |= 1u << i;
+      }
+    }
+    if (group_step) {
+      uint32_t kept = 0;
+      float Gs[16];
+#pragma unroll
+      for (int g = 0; g < 16; ++g) {
+        Gs[g] = -FLT_MAX;
+        if (g < p.n_group) {
+          float v1 = -FLT_MAX, v2 = -FLT_MAX;  // this lane's two largest c of group g
+#pragma unroll
+          for (int i = 0; i < W1_NE; ++i) {
+            if (gid[i] == g) {
+              if (c[i] > v1) {
+                v2 = v1;
+                v1 = c[i];
+              } else if (c[i] > v2) {
+                v2 = c[i];
+              }
+            }
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) {  // top-2 of the warp
+            const float o1 = __shfl_xor_sync(FULL, v1, off);
+            const float o2 = __shfl_xor_sync(FULL, v2, off);
+            const float hi = fmaxf(v1, o1), lo = fminf(v1, o1);
+            v2 = fmaxf(lo, fmaxf(v2, o2));
+            v1 = hi;
+          }
+          Gs[g] = v1 + v2;
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < 16; ++g) {  // larger score first, ties to the lower group
+        if (g < p.n_group) {
+          int rank = 0;
+#pragma unroll
+          for (int m = 0; m < 16; ++m)
+            if (m < p.n_group && (Gs[m] > Gs[g] || (Gs[m] == Gs[g] && m < g))) ++rank;
+          if (rank < p.topk_group) kept |= 1u << g;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < W1_NE; ++i)
+        if (gid[i] < 0 || !((kept >> gid[i]) & 1u)) avail &= ~(1u << i);
+    }
+    int my_id = -1;
+    float my_s = 0.f, sum = 0.f;
+    for (int r = 0; r < p.top_k; ++r) {
+      float v = -FLT_MAX;
+      int idx = INT_MAX;
+#pragma unroll
+      for (int i = 0; i < W1_NE; ++i)
+        if (((avail >> i) & 1u) && c[i] > v) {  // ascending ids: ties keep the lower
+          v = c[i];
+          idx = lane + 32 * i;
+        }
+      warp_argmax(v, idx);
+      const int slot = (idx >> 5) & (W1_NE - 1);
+      float sv = s[0];
+#pragma unroll
+      for (int i = 1; i < W1_NE; ++i)
+        if (slot == i) sv = s[i];
+      sv = __shfl_sync(FULL, sv, idx & 31);
+      if (idx < E) {
+        if (lane == (idx & 31)) avail &= ~(1u << slot);
+      } else {
+        sv = 0.f;
+        idx = -1;  // no candidate left (non-finite scores); the permutation reports it
+      }
+      sum += sv;
+      if (lane == r) {
+        my_id = idx;
+        my_s = sv;
+      }
+    }
+    if (lane < p.top_k) {
+      float wv = p.norm_topk_prob ? p.rsf * (my_s / sum) : p.rsf * my_s;
+      if (p.mask && p.mask[t] == 0) {  // padding token: no routed expert
+        my_id = -1;
+        wv = 0.f;
+      }
+      topk_ids[(size_t)t * p.top_k + lane] = my_id;
+      topk_w[(size_t)t * p.top_k + lane] = wv;
+    }
+  }
+}
+
 }  // namespace
 
 int router_splits(int H) {
@@ -444,11 +586,17 @@ cudaError_t launch_router(const void* x, const float* Wr, const float* bias, con
   err = launch_chained(router_gemm_kernel, dim3(grid), dim3(R_THREADS), R_SMEM_BYTES, stream, tmX,
                        tmW3, T, E, H / RBK, S, NP, partial, status, timeout_ns);
   if (err != cudaSuccess) return err;
-  int sel_grid = ((T + 1) / 2 + SEL_WARPS - 1) / SEL_WARPS;
-  const int cap = num_sms() * 16;
-  if (sel_grid > cap) sel_grid = cap;
-  err = launch_chained(router_select_kernel, dim3(sel_grid), dim3(SEL_WARPS * 32), 0, stream,
-                       (const float*)partial, S, bias, p, topk_ids, topk_w);
+  if (T <= ROUTER_WARP_SELECT_MAX_T) {  // small batches: one warp per token, short chains
+    const int grid = (T + 7) / 8;
+    err = launch_chained(router_select_warp_kernel, dim3(grid), dim3(256), 0, stream,
+                         (const float*)partial, S, bias, p, topk_ids, topk_w);
+  } else {
+    int sel_grid = ((T + 1) / 2 + SEL_WARPS - 1) / SEL_WARPS;
+    const int cap = num_sms() * 16;
+    if (sel_grid > cap) sel_grid = cap;
+    err = launch_chained(router_select_kernel, dim3(sel_grid), dim3(SEL_WARPS * 32), 0, stream,
+                         (const float*)partial, S, bias, p, topk_ids, topk_w);
+  }
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
