@@ -278,12 +278,12 @@ __global__ void __launch_bounds__(PT)
   }
 }
 
-// One warp per token: x[t] is read once (1 KB per warp step: 32 bytes per
-// lane) and written to the token's top_k rows with full-sector stores;
-// row_of gives the rows (-1: skipped id), fetched once per token.
+// One warp per token (small batches: several): x[t] is read once (1 KB per
+// warp step: 32 bytes per lane) and written to the token's top_k rows with
+// full-sector stores; row_of gives the rows (-1: skipped id), fetched once.
 __global__ void __launch_bounds__(256)
     gather_tokens_kernel(const __nv_bfloat16* __restrict__ x, const int* __restrict__ row_of,
-                         int T, int H, int top_k, __nv_bfloat16* __restrict__ xp) {
+                         int T, int H, int top_k, int parts, __nv_bfloat16* __restrict__ xp) {
   __shared__ int rows_sm[8][MAX_TOPK_PERMUTE];  // each warp's current token's rows
   pdl_launch_dependents();
   pdl_wait();
@@ -291,12 +291,15 @@ __global__ void __launch_bounds__(256)
   const int warps = gridDim.x * (blockDim.x >> 5);
   const int chunks = H / 16;  // 32-byte pieces of a row (H is a multiple of 64)
   int* rows = rows_sm[wib];
-  for (int t = blockIdx.x * (blockDim.x >> 5) + wib; t < T; t += warps) {
+  // `parts` warps share a token (small batches), each taking every parts-th
+  // 1 KB column block of the row
+  for (int wt = blockIdx.x * (blockDim.x >> 5) + wib; wt < T * parts; wt += warps) {
+    const int t = wt / parts, part = wt - t * parts;
     __syncwarp();  // the previous token's rows have been used
     if (lane < top_k) rows[lane] = row_of[(size_t)t * top_k + lane];
     __syncwarp();
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
-    for (int c = lane; c < chunks; c += 32) {
+    for (int c = lane + 32 * part; c < chunks; c += 32 * parts) {
       const uint4 a = src[2 * c], b = src[2 * c + 1];
       const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
       for (int j = 0; j < top_k; ++j) {
@@ -310,12 +313,19 @@ __global__ void __launch_bounds__(256)
 cudaError_t launch_gather(const void* x, int T, int H, int top_k, const PermuteOut& o,
                           cudaStream_t stream) {
   if (o.xp && x) {
-    int grid = (T + 7) / 8;
-    const int cap = num_sms() * 8;
+    // warps per token: enough warps to fill the GPU twice over, at most one
+    // per 1 KB column block of a row
+    const int cap = num_sms() * 8;  // blocks of 8 warps
+    int parts = (2 * cap * 8) / (T > 0 ? T : 1);
+    const int max_parts = H / 512;
+    if (parts > max_parts) parts = max_parts;
+    if (parts < 1) parts = 1;
+    long long grid = ((long long)T * parts + 7) / 8;
     if (grid > cap) grid = cap;
     const cudaError_t err = launch_chained(
-        gather_tokens_kernel, dim3(grid), dim3(256), 0, stream, static_cast<const __nv_bfloat16*>(x),
-        (const int*)o.row_of, T, H, top_k, static_cast<__nv_bfloat16*>(o.xp));
+        gather_tokens_kernel, dim3((unsigned)grid), dim3(256), 0, stream,
+        static_cast<const __nv_bfloat16*>(x), (const int*)o.row_of, T, H, top_k, parts,
+        static_cast<__nv_bfloat16*>(o.xp));
     if (err != cudaSuccess) return err;
   }
   return cudaGetLastError();
