@@ -26,4 +26,9 @@ from .moe_oracle import (  # noqa: F401
     moe_forward_tokens,
     permutation,
     rmsnorm,
+    FP8_BLOCK,
+    fp8_e4m3_decode,
+    ue8m0_decode,
+    fp8_block_dequant,
+    moe_forward_fp8,
 )

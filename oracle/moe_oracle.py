@@ -44,7 +44,9 @@ notes of the repository):
   * ``norm_topk_prob`` is on; the denominator has no epsilon guard;
   * ids are returned in selection order (descending c);
   * the padding mask is per token: a padding token takes no routed expert
-    (id -1, weight 0) and keeps the shared expert (see ``apply_token_mask``).
+    (id -1, weight 0) and keeps the shared expert (see ``apply_token_mask``);
+  * FP8 expert weights are E4M3 codes with one power-of-two scale per
+    128 x 128 block (see ``fp8_block_dequant``).
 """
 
 from __future__ import annotations
@@ -301,6 +303,64 @@ def moe_forward_tokens(tokens, x, Wr, bias, w13, w2, ws13, ws2, cfg: MoeConfig,
     sub_mask = None if token_mask is None else np.asarray(token_mask).reshape(-1)[tokens]
     return moe_forward(x[tokens], Wr, bias, w13, w2, ws13, ws2, cfg,
                        residual=res, ids=sub_ids, token_mask=sub_mask)
+
+
+# ----------------------------------------------------------------------------
+# FP8 expert weights.  [S3] "Known limitations" names an optional FP8 backend
+# of the upstream project and gives no format.  Reading: weight-only FP8 --
+# every expert matrix (routed and shared) stored as OCP E4M3 codes ("fn"
+# variant: no infinities) with one power-of-two scale per 128 x 128 block,
+# held as a UE8M0 exponent byte; activations, router and restore unchanged.
+# With power-of-two scales every dequantised weight is a bf16 value, so the
+# FP8 block is exactly the bf16 block evaluated on the dequantised weights.
+# ----------------------------------------------------------------------------
+FP8_BLOCK = 128
+
+
+def fp8_e4m3_decode(codes) -> np.ndarray:
+    """E4M3 codes (uint8) to float64, from the format's definition: sign bit 7,
+    exponent bits 6..3 (bias 7), mantissa bits 2..0.  Exponent 0 encodes
+    zero and the subnormals m/8 * 2^-6; exponent 15 with mantissa 7 is NaN;
+    every other code is (1 + m/8) * 2^(e-7) (largest: 448)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = c >> 7
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = np.where(sign == 1, -mag, mag)
+    return np.where((e == 15) & (m == 7), np.nan, val)
+
+
+def ue8m0_decode(exps) -> np.ndarray:
+    """UE8M0 scale bytes to float64: 2^(s - 127); 255 is NaN."""
+    s = np.asarray(exps, dtype=np.uint8).astype(np.float64)
+    return np.where(s == 255, np.nan, np.exp2(s - 127.0))
+
+
+def fp8_block_dequant(codes, scale_exp, block: int = FP8_BLOCK) -> np.ndarray:
+    """Dequantised weights, float64 [..., N, K]: element (n, k) of each matrix
+    is decode(codes[n, k]) * 2^(scale_exp[n // block, k // block] - 127).
+    ``scale_exp`` is [..., ceil(N/block), ceil(K/block)] (a partial last
+    block row / column has its own scale)."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    scale = ue8m0_decode(scale_exp)
+    N, K = codes.shape[-2], codes.shape[-1]
+    rows = np.arange(N) // block
+    cols = np.arange(K) // block
+    per_elem = scale[..., rows[:, None], cols[None, :]]
+    return fp8_e4m3_decode(codes) * per_elem
+
+
+def moe_forward_fp8(x, Wr, bias, w13_q, w13_s, w2_q, w2_s, ws13_q, ws13_s, ws2_q, ws2_s,
+                    cfg: MoeConfig, residual=None, ids=None, token_mask=None):
+    """``moe_forward`` with FP8 expert weights: each weight matrix is the
+    block dequantisation of its codes and scale exponents (``*_q`` uint8
+    codes shaped like the bf16 weights, ``*_s`` uint8 scale exponents per
+    128 x 128 block); everything else as ``moe_forward``."""
+    deq = lambda q, sc: None if q is None else fp8_block_dequant(q, sc)
+    return moe_forward(x, Wr, bias, deq(w13_q, w13_s), deq(w2_q, w2_s),
+                       deq(ws13_q, ws13_s), deq(ws2_q, ws2_s), cfg,
+                       residual=residual, ids=ids, token_mask=token_mask)
 
 
 # ----------------------------------------------------------------------------

@@ -15,6 +15,9 @@ are the fp32 draw rounded to nearest-even by ``Tensor.to(torch.bfloat16)``.
   w2    ~ N(0, 0.02)       bf16 [E, H, I]
   ws13  ~ N(0, 0.02)       bf16 [2I_s, H]
   ws2   ~ N(0, 0.02)       bf16 [H, I_s]
+FP8 expert weights (``make_fp8_weights``): the same normal draws as w13..ws2,
+stored as E4M3 codes with one power-of-two scale per 128 x 128 block
+(scale exponents: tensor indices 7-10).
 """
 
 from __future__ import annotations
@@ -119,6 +122,46 @@ def make_dense_weights(H: int, I: int, seed: int, device="cpu", std: float = 0.0
     base = seed * 1000
     return dict(w13=_normal((2 * I, H), std, base + 3, device, torch.bfloat16),
                 w2=_normal((H, I), std, base + 4, device, torch.bfloat16))
+
+
+FP8_BLOCK = 128  # rows and columns of one scale block of an FP8 weight matrix
+
+
+def _fp8_matrix(shape, std, seed, scale_seed, device):
+    """E4M3 codes (uint8, ``shape``) and UE8M0 scale exponents (uint8, one per
+    128 x 128 block of the last two dimensions): exponents ~ U{118, 119, 120}
+    (scales 2^-9 .. 2^-7); codes = the N(0, std) draw of seed ``seed`` divided by
+    its block's scale, clamped to +-448 and cast by ``Tensor.to(float8_e4m3fn)``."""
+    N, K = shape[-2], shape[-1]
+    nb, kb = -(-N // FP8_BLOCK), -(-K // FP8_BLOCK)
+    sexp = torch.randint(118, 121, (*shape[:-2], nb, kb), generator=_gen(scale_seed, device),
+                         device=device, dtype=torch.int32)
+    scale = torch.exp2(sexp.to(torch.float32) - 127.0)
+    scale = scale.repeat_interleave(FP8_BLOCK, -2)[..., :N, :]
+    scale = scale.repeat_interleave(FP8_BLOCK, -1)[..., :K]
+    draw = _normal(shape, std, seed, device, torch.float32)
+    codes = (draw / scale).clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes, sexp.to(torch.uint8)
+
+
+def make_fp8_weights(H: int, seed: int, E: int = 128, I: int = 768, I_shared: int = 768,
+                     device="cpu", layer: int = 0, w13_std: float = 0.02,
+                     w2_std: float = 0.02):
+    """FP8 expert weights of one block: dict(w13_q, w13_s, w2_q, w2_s, ws13_q,
+    ws13_s, ws2_q, ws2_s); ``*_q`` E4M3 codes shaped like the bf16 weights of
+    ``make_weights``, drawn from the same normal draws (tensor indices 3-6),
+    ``*_s`` their UE8M0 block scale exponents (tensor indices 7-10)."""
+    base = seed * 1000 + 100 * layer
+    d = {}
+    d["w13_q"], d["w13_s"] = _fp8_matrix((E, 2 * I, H), w13_std, base + 3, base + 7, device)
+    d["w2_q"], d["w2_s"] = _fp8_matrix((E, H, I), w2_std, base + 4, base + 8, device)
+    if I_shared > 0:
+        d["ws13_q"], d["ws13_s"] = _fp8_matrix((2 * I_shared, H), w13_std, base + 5, base + 9,
+                                               device)
+        d["ws2_q"], d["ws2_s"] = _fp8_matrix((H, I_shared), w2_std, base + 6, base + 10, device)
+    else:
+        d["ws13_q"] = d["ws13_s"] = d["ws2_q"] = d["ws2_s"] = None
+    return d
 
 
 def make_block_inputs(T: int, H: int, seed: int, E: int = 128, I: int = 768,

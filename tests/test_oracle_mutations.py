@@ -5,6 +5,7 @@ import numpy as np
 import pytest
 
 import oracle.moe_oracle as om
+from tests import test_oracle_fp8 as fp8_pins
 from tests import test_oracle_pins as pins
 
 
@@ -78,6 +79,37 @@ def _forward_mask_kills_shared(*args, **kw):
         out[pad] = 0.0 if res is None else np.asarray(res, dtype=np.float64)[pad]
     return out, ids, w, m
 
+def _e4m3_bias_8(codes):
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    e, m = (c >> 3) & 0xF, c & 7
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -7, (1.0 + m / 8.0) * np.exp2(e - 8.0))
+    val = np.where(c >> 7 == 1, -mag, mag)
+    return np.where((e == 15) & (m == 7), np.nan, val)
+
+
+def _e4m3_subnormals_as_normals(codes):
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    e, m = (c >> 3) & 0xF, c & 7
+    mag = (1.0 + m / 8.0) * np.exp2(e - 7.0)
+    val = np.where(c >> 7 == 1, -mag, mag)
+    return np.where((e == 15) & (m == 7), np.nan, val)
+
+
+def _ue8m0_bias_128(exps):
+    s = np.asarray(exps, dtype=np.uint8).astype(np.float64)
+    return np.where(s == 255, np.nan, np.exp2(s - 128.0))
+
+
+def _block_index_transposed(codes, scale_exp, block=128):
+    # row block and column block swapped in the scale lookup (on a non-square
+    # block grid this reads the wrong scales or runs off the grid)
+    codes = np.asarray(codes, dtype=np.uint8)
+    scale = om.ue8m0_decode(scale_exp)
+    rows = np.arange(codes.shape[-2]) // block
+    cols = np.arange(codes.shape[-1]) // block
+    return om.fp8_e4m3_decode(codes) * scale[..., cols[None, :], rows[:, None]]
+
+
 PIN_TESTS = [
     lambda: pins.test_hand_worked_golden_example(),
     lambda: [pins.test_selection_matches_brute_force(*a) for a in
@@ -88,6 +120,9 @@ PIN_TESTS = [
     lambda: pins.test_single_expert_is_textbook_swiglu_plus_shared(),
     lambda: pins.test_swiglu_gate_up_order_and_w2_orientation(),
     lambda: pins.test_padding_mask_keeps_only_the_shared_expert(),
+    lambda: fp8_pins.test_e4m3_decode_matches_torch_float8_on_every_code(),
+    lambda: fp8_pins.test_ue8m0_scales(),
+    lambda: fp8_pins.test_block_scales_land_on_their_blocks_ragged_non_square(),
 ]
 
 MUTATIONS = {
@@ -106,6 +141,14 @@ MUTATIONS = {
     "shared_expert_scaled": [(pins, "moe_forward", _scaled_shared)],
     "padding_mask_ignored": [(om, "apply_token_mask", _mask_ignored)],
     "padding_drops_shared_expert": [(pins, "moe_forward", _forward_mask_kills_shared)],
+    "e4m3_exponent_bias_8": [(om, "fp8_e4m3_decode", _e4m3_bias_8),
+                             (fp8_pins, "fp8_e4m3_decode", _e4m3_bias_8)],
+    "e4m3_subnormals_as_normals": [(om, "fp8_e4m3_decode", _e4m3_subnormals_as_normals),
+                                   (fp8_pins, "fp8_e4m3_decode", _e4m3_subnormals_as_normals)],
+    "ue8m0_bias_128": [(om, "ue8m0_decode", _ue8m0_bias_128),
+                       (fp8_pins, "ue8m0_decode", _ue8m0_bias_128)],
+    "fp8_block_index_transposed": [(om, "fp8_block_dequant", _block_index_transposed),
+                                   (fp8_pins, "fp8_block_dequant", _block_index_transposed)],
 }
 
 
