@@ -208,6 +208,32 @@ MOE_API int32_t moe_forward(const void* x, const float* Wr, const float* bias, c
                     void* out, const moe_forward_opts_t* opts, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/* moe_forward with FP8 expert weights.  The pages name an optional FP8
+ * backend of the upstream project ([S3] "Known limitations") without a
+ * format; this entry point takes weight-only FP8: every expert matrix as OCP
+ * E4M3 codes ("fn": no infinities) with one power-of-two scale per 128 x 128
+ * block, given as a UE8M0 byte s (scale 2^(s-127)).  Weights are dequantised
+ * to bf16 in shared memory next to the tensor cores; with power-of-two
+ * scales the dequantised weights are exact bf16 values, so the result is bit
+ * for bit that of moe_forward on the dequantised bf16 weights.
+ *   w13_q  device uint8 [E,2I,H]  E4M3 codes, gate rows then up rows
+ *   w13_s  device uint8 [E,2I/128,H/128]  scale exponents
+ *   w2_q   device uint8 [E,H,I];  w2_s device uint8 [E,H/128,I/128]
+ *   ws13_q / ws13_s  [2I_s,H] / [2I_s/128,H/128];  ws2_q / ws2_s  [H,I_s] /
+ *          [H/128,I_s/128]  the shared expert (NULL when I_shared == 0)
+ * H, I and I_shared must be multiples of 128 (MOE_ERR_UNSUPPORTED_SHAPE);
+ * scale exponents 255 (NaN) and E4M3 NaN codes are not checked and give
+ * undefined values.  Workspace: moe_workspace_bytes(cfg).  Every other
+ * argument, option and error as moe_forward.  The expert GEMMs run with
+ * swapped operands (weight rows on the MMA's M) at every batch size. */
+MOE_API int32_t moe_forward_fp8(const void* x, const float* Wr, const float* bias,
+                                const uint8_t* w13_q, const uint8_t* w13_s,
+                                const uint8_t* w2_q, const uint8_t* w2_s,
+                                const uint8_t* ws13_q, const uint8_t* ws13_s,
+                                const uint8_t* ws2_q, const uint8_t* ws2_s,
+                                const moe_cfg_t* cfg, void* out, const moe_forward_opts_t* opts,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
 /* Workspace bytes of moe_forward_host: those of moe_forward plus four
  * [T,H] bf16 staging buffers (two for inputs, two for outputs); 0 for an
  * invalid configuration. */

@@ -440,6 +440,190 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
   return MOE_OK;
 }
 
+// The expert and shared-expert GEMMs with FP8 weights: the swapped kernels
+// with weight tiles dequantised in shared memory (grouped_gemm_swap_fp8.cu).
+struct Fp8Weights {
+  const uint8_t *w13_q, *w13_s, *w2_q, *w2_s, *ws13_q, *ws13_s, *ws2_q, *ws2_s;
+};
+
+template <typename Rec>
+cudaError_t swap_gemms_fp8(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp,
+                           __nv_bfloat16* h, __nv_bfloat16* hs, __nv_bfloat16* Y,
+                           const Fp8Weights& fw, const int* offsets, const PermuteOut& o,
+                           const GemmArgs& a, int sms, Rec& record, cudaStream_t s) {
+  const size_t T = c.T, R = T * c.top_k;
+  const int slots = slots_per_token(c);
+  const bool fused = fuse_shared(c);
+  const int groups = c.E + (fused ? 1 : 0);
+  const int chunk = swap_chunk(c);
+  const long long chunk_bound = (long long)(R / chunk) + groups + 1;
+  const size_t h_rows = R + (fused ? T : 0);
+  CUtensorMap tm_xp, tm_x, tm_h, tm_hs, tm_w13, tm_w2, tm_ws13, tm_ws2;
+  cudaError_t e;
+  if ((e = make_tmap_2d_box(&tm_xp, xp, R, c.H, 32)) != cudaSuccess) return e;
+  if ((e = make_tmap_2d_box(&tm_h, h, h_rows, c.I, 32)) != cudaSuccess) return e;
+  if ((e = make_tmap_3d_fp8(&tm_w13, fw.w13_q, c.E, 2 * (uint64_t)c.I, c.H)) != cudaSuccess)
+    return e;
+  if ((e = make_tmap_3d_fp8(&tm_w2, fw.w2_q, c.E, c.H, c.I)) != cudaSuccess) return e;
+  tm_x = tm_hs = tm_xp;  // unused unless there is a shared expert
+  tm_ws13 = tm_w13;
+  tm_ws2 = tm_w2;
+  if (c.I_shared > 0) {
+    if ((e = make_tmap_2d_box(&tm_x, x, T, c.H, 32)) != cudaSuccess) return e;
+    if (!fused && (e = make_tmap_2d_box(&tm_hs, hs, T, c.I_shared, 32)) != cudaSuccess) return e;
+    if ((e = make_tmap_3d_fp8(&tm_ws13, fw.ws13_q, 1, 2 * (uint64_t)c.I_shared, c.H)) !=
+        cudaSuccess)
+      return e;
+    if ((e = make_tmap_3d_fp8(&tm_ws2, fw.ws2_q, 1, c.H, c.I_shared)) != cudaSuccess) return e;
+  }
+  const Fp8Scales up_sc{fw.w13_s, fw.ws13_s, 2 * c.I / 128, c.H / 128};
+  const Fp8Scales down_sc{fw.w2_s, fw.ws2_s, c.H / 128, c.I / 128};
+  if ((e = record(MOE_STAGE_EXPERT_UP)) != cudaSuccess) return e;
+  {  // h[r, i] = silu(W13g[i] . x_r) * (W13u[i] . x_r) per group (shared expert: group E)
+    GemmArgs g = a;
+    g.mtile_start = o.mtile_start;
+    g.row_start = offsets;
+    g.num_groups = groups;
+    if (fused) {
+      g.alt_group = c.E;
+      g.alt_rebase = 1;
+    }
+    g.n_tiles = c.I / 128;
+    g.k_steps = c.H / 64;
+    g.n_out_tile = 128;
+    g.b_second = c.I;
+    g.out = h;
+    g.ldo = c.I;
+    g.n_valid = c.I;
+    const int grid = (int)std::min<long long>(sms, chunk_bound * g.n_tiles);
+    if ((e = launch_grouped_gemm_swap_fp8(EPI_SWIGLU, chunk, tm_w13, tm_xp, tm_ws13, tm_x, g,
+                                          up_sc, grid, s)) != cudaSuccess)
+      return e;
+  }
+  if ((e = record(MOE_STAGE_EXPERT_DOWN)) != cudaSuccess) return e;
+  {  // Y[pos_r, n] = w_r * (W2[n] . h_r) per expert; shared rows to slot top_k, unscaled
+    GemmArgs g = a;
+    g.mtile_start = o.mtile_start;
+    g.row_start = offsets;
+    g.num_groups = groups;
+    if (fused) {
+      g.alt_group = c.E;
+      g.alt_rebase = 0;
+    }
+    g.n_tiles = c.H / 128;
+    g.k_steps = c.I / 64;
+    g.n_out_tile = 128;
+    g.out = Y;
+    g.ldo = c.H;
+    g.n_valid = c.H;
+    g.row_scale = o.w_of;
+    g.dest_pos = o.pos_of;
+    g.dest_mul = slots;
+    g.dest_add = c.top_k;
+    const int grid = (int)std::min<long long>(sms, chunk_bound * g.n_tiles);
+    if ((e = launch_grouped_gemm_swap_fp8(EPI_ROWSCALE, chunk, tm_w2, tm_h, tm_ws2, tm_h, g,
+                                          down_sc, grid, s)) != cudaSuccess)
+      return e;
+  }
+  if ((e = record(MOE_STAGE_SHARED_EXPERT)) != cudaSuccess) return e;
+  if (c.I_shared > 0 && !fused) {
+    const long long chunks = (long long)(T + chunk - 1) / chunk;
+    {  // hs = silu(x . Ws13g^T) * (x . Ws13u^T)
+      GemmArgs g = a;
+      g.single_rows = c.T;
+      g.n_tiles = c.I_shared / 128;
+      g.k_steps = c.H / 64;
+      g.n_out_tile = 128;
+      g.b_second = c.I_shared;
+      g.out = hs;
+      g.ldo = c.I_shared;
+      g.n_valid = c.I_shared;
+      const Fp8Scales sc{fw.ws13_s, nullptr, 2 * c.I_shared / 128, c.H / 128};
+      const int grid = (int)std::min<long long>(sms, chunks * g.n_tiles);
+      if ((e = launch_grouped_gemm_swap_fp8(EPI_SWIGLU, chunk, tm_ws13, tm_x, tm_ws13, tm_x, g,
+                                            sc, grid, s)) != cudaSuccess)
+        return e;
+    }
+    {  // Y[t*slots + top_k] = hs . Ws2^T  (unscaled)
+      GemmArgs g = a;
+      g.single_rows = c.T;
+      g.n_tiles = c.H / 128;
+      g.k_steps = c.I_shared / 64;
+      g.n_out_tile = 128;
+      g.out = Y;
+      g.ldo = c.H;
+      g.n_valid = c.H;
+      g.dest_mul = slots;
+      g.dest_add = c.top_k;
+      const Fp8Scales sc{fw.ws2_s, nullptr, c.H / 128, c.I_shared / 128};
+      const int grid = (int)std::min<long long>(sms, chunks * g.n_tiles);
+      if ((e = launch_grouped_gemm_swap_fp8(EPI_ROWSCALE, chunk, tm_ws2, tm_hs, tm_ws2, tm_hs, g,
+                                            sc, grid, s)) != cudaSuccess)
+        return e;
+    }
+  }
+  return cudaSuccess;
+}
+
+// The launch sequence of the block forward with FP8 expert weights: the
+// router, permutation and combine of forward_impl around swap_gemms_fp8.
+int32_t forward_fp8_impl(const void* x, const float* Wr, const float* bias, const Fp8Weights& fw,
+                         const moe_cfg_t& c, void* out, const moe_forward_opts_t* opts,
+                         void* workspace, cudaStream_t s) {
+  const FwdLayout L = fwd_layout(c);
+  void** ev = opts ? opts->stage_events : nullptr;
+  const unsigned long long timeout =
+      (opts && opts->wait_timeout_ns > 0) ? (unsigned long long)opts->wait_timeout_ns
+                                          : DEFAULT_TIMEOUT_NS;
+  int* status = at<int>(workspace, L.status);
+  int32_t* ids = (opts && opts->topk_ids) ? opts->topk_ids : at<int32_t>(workspace, L.ids);
+  float* tw = (opts && opts->topk_w) ? opts->topk_w : at<float>(workspace, L.w);
+  int* offsets = at<int>(workspace, L.offsets);
+  int* row_of = at<int>(workspace, L.row_of);
+  __nv_bfloat16* xp = at<__nv_bfloat16>(workspace, L.y);
+  __nv_bfloat16* Y = xp;
+  __nv_bfloat16* h = at<__nv_bfloat16>(workspace, L.h);
+  __nv_bfloat16* hs = at<__nv_bfloat16>(workspace, L.hs);
+  const int slots = slots_per_token(c);
+  const bool fused = fuse_shared(c);
+  const int sms = num_sms();
+  auto record = [&](int i) -> cudaError_t {
+    return (ev && ev[i]) ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
+  };
+
+  RMOE_TRY(record(MOE_STAGE_ROUTER));
+  RouterParams rp = router_params(c);
+  rp.mask = opts ? opts->token_mask : nullptr;
+  RMOE_TRY(launch_router(x, Wr, bias, rp, ids, tw, at<void>(workspace, L.router), status, timeout,
+                         s));
+  RMOE_TRY(record(MOE_STAGE_PERMUTE));
+  PermuteOut o;
+  o.status = status;
+  o.blk_hist = at<int>(workspace, L.blk_hist);
+  o.expert_offsets = offsets;
+  o.mtile_start = at<int>(workspace, L.mtiles);
+  o.row_of = row_of;
+  o.tok_of = at<int>(workspace, L.tok_of);
+  o.w_of = at<float>(workspace, L.w_of);
+  o.pos_of = at<int>(workspace, L.pos_of);
+  o.slot_stride = slots;
+  o.extra_rows = fused ? c.T : 0;
+  o.xp = xp;
+  o.mask = rp.mask;
+  RMOE_TRY(launch_permute(ids, tw, x, c.T, c.H, c.E, c.top_k, o, s));
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.status = status;
+  a.timeout_ns = timeout;
+  a.alt_group = -1;
+  RMOE_TRY(swap_gemms_fp8(c, x, xp, h, hs, Y, fw, offsets, o, a, sms, record, s));
+  RMOE_TRY(record(MOE_STAGE_COMBINE));
+  const void* residual = opts ? opts->residual : nullptr;
+  RMOE_TRY(launch_combine_slots(Y, row_of, c.top_k, c.T, c.H, slots, residual, out, s));
+  RMOE_TRY(record(MOE_NUM_STAGES));
+  return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -538,6 +722,28 @@ int32_t moe_forward(const void* x, const float* Wr, const float* bias, const voi
   if (!ws_ok(workspace, workspace_bytes, fwd_layout(c).total)) return MOE_ERR_WORKSPACE;
   return forward_impl(x, Wr, bias, w13, w2, ws13, ws2, c, out, opts, workspace, true,
                       static_cast<cudaStream_t>(stream));
+}
+
+int32_t moe_forward_fp8(const void* x, const float* Wr, const float* bias, const uint8_t* w13_q,
+                        const uint8_t* w13_s, const uint8_t* w2_q, const uint8_t* w2_s,
+                        const uint8_t* ws13_q, const uint8_t* ws13_s, const uint8_t* ws2_q,
+                        const uint8_t* ws2_s, const moe_cfg_t* cfg, void* out,
+                        const moe_forward_opts_t* opts, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  const int32_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  const moe_cfg_t& c = *cfg;
+  if (c.H % 128 != 0 || c.I % 128 != 0 || c.I_shared % 128 != 0)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (c.T == 0) return MOE_OK;
+  if (!w13_s || !w2_s) return MOE_ERR_INVALID_ARG;
+  if ((c.I_shared > 0) != (ws13_s != nullptr && ws2_s != nullptr)) return MOE_ERR_INVALID_ARG;
+  const int32_t a = check_forward_args(c, x, Wr, bias, w13_q, w2_q, ws13_q, ws2_q, out, opts);
+  if (a != MOE_OK) return a;
+  if (!ws_ok(workspace, workspace_bytes, fwd_layout(c).total)) return MOE_ERR_WORKSPACE;
+  const Fp8Weights fw{w13_q, w13_s, w2_q, w2_s, ws13_q, ws13_s, ws2_q, ws2_s};
+  return forward_fp8_impl(x, Wr, bias, fw, c, out, opts, workspace,
+                          static_cast<cudaStream_t>(stream));
 }
 
 size_t moe_forward_host_workspace_bytes(const moe_cfg_t* cfg) {

@@ -123,6 +123,28 @@ cudaError_t launch_grouped_gemm_swap(int epi, int chunk, const CUtensorMap& tmW,
                                      const CUtensorMap& tmX2, const GemmArgs& args, int grid,
                                      cudaStream_t stream);
 
+// FP8 expert weights (grouped_gemm_swap_fp8.cu): UE8M0 scale exponents, one
+// per 128 x 128 block, [groups][rows][cols] for the routed experts (s) and
+// [rows][cols] for the group args.alt_group (s2); cols = K / 128.
+struct Fp8Scales {
+  const uint8_t* s;
+  const uint8_t* s2;
+  int rows;  // scale-block rows per group of s
+  int cols;  // scale-block columns (K / 128)
+};
+
+// 3D map over [groups, N_rows, K] E4M3 codes (bytes), box 128 x 128 x 1, 128B swizzle.
+cudaError_t make_tmap_3d_fp8(CUtensorMap* map, const void* base, uint64_t groups, uint64_t n_rows,
+                             uint64_t K);
+
+// The swapped grouped GEMM with FP8 weights: as launch_grouped_gemm_swap, with
+// tmW / tmW2 E4M3 maps (make_tmap_3d_fp8) and their block scales in sc; K and
+// the weight-row offsets (args.b_second) must be multiples of 128.
+cudaError_t launch_grouped_gemm_swap_fp8(int epi, int chunk, const CUtensorMap& tmW,
+                                         const CUtensorMap& tmX, const CUtensorMap& tmW2,
+                                         const CUtensorMap& tmX2, const GemmArgs& args,
+                                         const Fp8Scales& sc, int grid, cudaStream_t stream);
+
 int num_sms();
 
 // ------------------------------------------------------------------ misc

@@ -95,6 +95,8 @@ def lib() -> ctypes.CDLL:
         "moe_permute": (i32, [vp, vp, vp, cfgp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "moe_forward": (i32, [vp, vp, vp, vp, vp, vp, vp, cfgp, vp,
                               ctypes.POINTER(MoeForwardOpts), vp, sz, vp]),
+        "moe_forward_fp8": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, cfgp, vp,
+                                  ctypes.POINTER(MoeForwardOpts), vp, sz, vp]),
         "moe_forward_host_workspace_bytes": (sz, [cfgp]),
         "moe_forward_host": (i32, [ctypes.POINTER(vp), ctypes.POINTER(vp), i32, vp, vp, vp, vp,
                                    vp, vp, cfgp, vp, sz, vp, vp, vp]),
@@ -282,6 +284,64 @@ def forward(x: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor, w13: torch.Te
     _check(lib().moe_forward(_ptr(x), _ptr(Wr), _ptr(bias), _ptr(w13), _ptr(w2), _ptr(ws13),
                              _ptr(ws2), ctypes.byref(c), _ptr(out), ctypes.byref(opts),
                              _ptr(workspace), workspace.numel(), _stream_ptr()), "moe_forward")
+    return out
+
+
+def forward_fp8(x: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor, fp8: dict,
+                cfg: BlockConfig, residual: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+                timer: Optional[StageTimer] = None, wait_timeout_ns: int = 0,
+                token_mask: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Block forward with FP8 expert weights (E4M3 codes, one power-of-two
+    scale per 128 x 128 block); returns out bf16 [T,H].  ``fp8`` holds uint8
+    tensors w13_q [E,2I,H], w13_s [E,2I/128,H/128], w2_q [E,H,I],
+    w2_s [E,H/128,I/128] and, with a shared expert, ws13_q, ws13_s, ws2_q,
+    ws2_s (the layouts of moe_forward_fp8)."""
+    T, H, E, I, Is = cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared
+    u8 = torch.uint8
+    _need(x, "x", torch.bfloat16, (T, H))
+    _need(Wr, "Wr", torch.float32, (E, H))
+    _need(bias, "bias", torch.float32, (E,))
+    blk = lambda n: -(-n // 128)
+    _need(fp8["w13_q"], "w13_q", u8, (E, 2 * I, H))
+    _need(fp8["w13_s"], "w13_s", u8, (E, blk(2 * I), blk(H)))
+    _need(fp8["w2_q"], "w2_q", u8, (E, H, I))
+    _need(fp8["w2_s"], "w2_s", u8, (E, blk(H), blk(I)))
+    shared = [None] * 4
+    if Is > 0:
+        _need(fp8["ws13_q"], "ws13_q", u8, (2 * Is, H))
+        _need(fp8["ws13_s"], "ws13_s", u8, (blk(2 * Is), blk(H)))
+        _need(fp8["ws2_q"], "ws2_q", u8, (H, Is))
+        _need(fp8["ws2_s"], "ws2_s", u8, (blk(H), blk(Is)))
+        shared = [fp8["ws13_q"], fp8["ws13_s"], fp8["ws2_q"], fp8["ws2_s"]]
+    if residual is not None:
+        _need(residual, "residual", torch.bfloat16, (T, H))
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    else:
+        _need(out, "out", torch.bfloat16, (T, H))
+    if topk_ids is not None:
+        _need(topk_ids, "topk_ids", torch.int32, (T, cfg.top_k))
+    if topk_w is not None:
+        _need(topk_w, "topk_w", torch.float32, (T, cfg.top_k))
+    if token_mask is not None:
+        _need(token_mask, "token_mask", torch.uint8, (T,))
+    if workspace is None:
+        workspace = alloc_workspace(workspace_bytes(cfg), x.device)
+    opts = MoeForwardOpts(
+        residual=None if residual is None else residual.data_ptr(),
+        topk_ids=None if topk_ids is None else topk_ids.data_ptr(),
+        topk_w=None if topk_w is None else topk_w.data_ptr(),
+        stage_events=timer.as_ptr() if timer is not None else None,
+        wait_timeout_ns=int(wait_timeout_ns),
+        token_mask=None if token_mask is None else token_mask.data_ptr())
+    c = cfg.c()
+    _check(lib().moe_forward_fp8(
+        _ptr(x), _ptr(Wr), _ptr(bias), _ptr(fp8["w13_q"]), _ptr(fp8["w13_s"]),
+        _ptr(fp8["w2_q"]), _ptr(fp8["w2_s"]), *[_ptr(t) for t in shared], ctypes.byref(c),
+        _ptr(out), ctypes.byref(opts), _ptr(workspace), workspace.numel(), _stream_ptr()),
+        "moe_forward_fp8")
     return out
 
 

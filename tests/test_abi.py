@@ -189,3 +189,29 @@ def test_dense_ffn_rejects_bad_arguments_on_the_host(L):
     assert L.moe_dense_ffn(*args(nbytes=need - 1)) == 3
     assert L.moe_dense_ffn(*args(ws=ctypes.c_void_p(0x10010))) == 3
     assert L.moe_dense_ffn(*args(T=0, x=None, out=None)) == 0
+
+
+def test_forward_fp8_rejects_bad_arguments_on_the_host(L):
+    c = BlockConfig(T=64, H=256, I=128, I_shared=128).c()
+    need = L.moe_workspace_bytes(ctypes.byref(c))
+    out = ctypes.c_void_p(0x20000)
+
+    def call(cfg=c, x=FAKE, q=(FAKE,) * 8, o=out, ws=FAKE, nbytes=need):
+        return L.moe_forward_fp8(x, FAKE, FAKE, *q, ctypes.byref(cfg), o, None, ws, nbytes,
+                                 None)
+
+    assert call(x=None) == 1
+    assert call(q=(FAKE, None) + (FAKE,) * 6) == 1            # w13 scales missing
+    assert call(q=(FAKE,) * 4 + (None,) * 4) == 1             # shared weights missing
+    assert call(q=(FAKE,) * 6 + (None, FAKE)) == 1            # shared w2 codes missing
+    assert call(o=FAKE) == 1                                  # out aliases x
+    assert call(nbytes=need - 1) == 3
+    assert call(ws=ctypes.c_void_p(0x10010)) == 3
+    # H, I and I_shared must be multiples of the 128-wide scale blocks
+    for bad in (BlockConfig(T=64, H=320, I=128, I_shared=128),
+                BlockConfig(T=64, H=256, I=192, I_shared=192),
+                BlockConfig(T=64, H=256, I=128, I_shared=64)):
+        assert call(cfg=bad.c()) == 2
+    assert call(cfg=BlockConfig(T=64, H=250).c()) == 2
+    z = BlockConfig(T=0, H=256, I=128, I_shared=128).c()
+    assert call(cfg=z, x=None, q=(None,) * 8, o=None, ws=None, nbytes=0) == 0
