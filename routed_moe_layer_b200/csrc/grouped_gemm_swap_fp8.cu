@@ -529,13 +529,11 @@ __global__ void __launch_bounds__(THREADS, 1)
               uint4* d1 = reinterpret_cast<uint4*>(row + (((j0 + 1) ^ sw) << 4));
               const uint4 lo = make_uint4(o[0], o[1], o[2], o[3]);
               const uint4 hi = make_uint4(o[4], o[5], o[6], o[7]);
-              if (odd_first) {
-                *d1 = hi;
-                *d0 = lo;
-              } else {
-                *d0 = lo;
-                *d1 = hi;
-              }
+              // selects, not a branch: all 32 lanes issue each of the two stores
+              uint4* const first = odd_first ? d1 : d0;
+              uint4* const second = odd_first ? d0 : d1;
+              *first = odd_first ? hi : lo;
+              *second = odd_first ? lo : hi;
             }
           }
           fence_proxy_async_smem();
