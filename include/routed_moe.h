@@ -292,6 +292,58 @@ MOE_API int32_t moe_dense_ffn(const void* x, const void* w13, const void* w2, in
                               int32_t H, int32_t I, const void* residual, void* out,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------- expert parallelism
+ * Building blocks of the block with its experts split across ranks (one GPU
+ * per rank): every rank routes and permutes its own tokens (moe_route,
+ * moe_permute: the rows for each rank's experts are then contiguous), sends
+ * the rows, their expert ids (moe_rows_expert_ids) and router weights to the
+ * ranks that hold those experts, which sort them by expert (moe_permute with
+ * top_k = 1) and run moe_expert_rows; the results come back to the tokens'
+ * ranks, which restore each token with moe_combine_rows and the shared expert
+ * (moe_dense_ffn on their own tokens).  The exchange itself is the caller's
+ * (an all-to-all each way).  The arithmetic of every row and of the restore is
+ * the block's own ([S1] LingBotVideoSparseMoeBlock.forward; [S2] the fp32
+ * restore), so the result is bit for bit that of moe_forward; the pages state
+ * no expert-parallel form ([S3] "Known limitations": no expert parallelism is
+ * claimed), and this split is the library's own. */
+
+/* ids[r] (device int32 [R]) = the expert e whose rows [offsets[e], offsets[e+1])
+ * contain row offsets[0] + r; offsets device int32 [E+1], non-decreasing,
+ * R = offsets[E] - offsets[0].  E in 1..128. */
+MOE_API int32_t moe_rows_expert_ids(const int32_t* offsets, int32_t E, int32_t R, int32_t* ids,
+                                    void* stream);
+
+/* Workspace bytes of moe_expert_rows; 0 for invalid sizes. */
+MOE_API size_t moe_expert_rows_workspace_bytes(int32_t R, int32_t H, int32_t E, int32_t I);
+
+/* The routed experts on rows already grouped by expert: for expert e (0..E-1)
+ * and each row r in [offsets[e], offsets[e+1]):
+ *   y[row_dest[r]] = bf16( row_w[r] * (silu(x_r.Wg_e^T) * (x_r.Wu_e^T)) . W2_e^T )
+ * with h stored in bf16 and the weight applied in fp32, as in moe_forward.
+ *   xr       device bf16 [R,H]; offsets device int32 [E+1], offsets[0] >= 0,
+ *            offsets[E] <= R (rows outside the groups are not computed)
+ *   w13      device bf16 [E,2I,H] (gate rows, then up rows); w2 device bf16 [E,H,I]
+ *   row_w    device fp32 [R] (NULL: 1); row_dest device int32 [R], distinct rows of y
+ *   y        device bf16 [>= max(row_dest)+1, H]
+ * E in 1..128; H and I multiples of 64 (<= 16384).  Workspace:
+ * moe_expert_rows_workspace_bytes(R,H,E,I), 256-byte aligned; device-side errors
+ * go to its status word (moe_read_device_status). */
+MOE_API int32_t moe_expert_rows(const void* xr, const int32_t* offsets, int32_t R, int32_t E,
+                                int32_t H, int32_t I, const void* w13, const void* w2,
+                                const float* row_w, const int32_t* row_dest, void* y,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* The restore with each token's routed rows addressed through row_of:
+ *   out[t] = bf16( sum_{j<top_k} y[row_of[t*top_k+j]] [+ shared[t]] [+ residual[t]] )
+ * summed in fp32 in that order (a row_of entry < 0 adds 0), rounded once -- the
+ * order and rounding of moe_forward's restore ([S2] "_restore_tokens").
+ *   y device bf16 [rows,H]; row_of device int32 [T,top_k]; shared, residual
+ *   device bf16 [T,H] or NULL; out device bf16 [T,H] (may be residual).
+ * H a multiple of 64 (<= 16384); top_k in 1..16. */
+MOE_API int32_t moe_combine_rows(const void* y, const int32_t* row_of, int32_t T, int32_t H,
+                                 int32_t top_k, const void* shared, const void* residual,
+                                 void* out, void* stream);
+
 /* RMSNorm with fp32 accumulation ([S2]: RMSNorm accumulates in fp32), for a
  * residual stack of blocks: xn = bf16(x * rsqrt(mean(x^2) + eps) * gamma).
  *   x device bf16 [T,H]; gamma device fp32 [H] or NULL (= 1); xn device bf16 [T,H]. */

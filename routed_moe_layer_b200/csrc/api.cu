@@ -897,6 +897,107 @@ int32_t moe_dense_ffn(const void* x, const void* w13, const void* w2, int32_t T,
   return MOE_OK;
 }
 
+int32_t moe_rows_expert_ids(const int32_t* offsets, int32_t E, int32_t R, int32_t* ids,
+                            void* stream) {
+  if (E <= 0 || E > MAX_E || R < 0) return MOE_ERR_INVALID_ARG;
+  if (R == 0) return MOE_OK;
+  if (!offsets || !ids) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_rows_expert_ids(offsets, E, R, ids, static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_expert_rows_workspace_bytes(int32_t R, int32_t H, int32_t E, int32_t I) {
+  if (R < 0 || E <= 0 || E > MAX_E || H <= 0 || I <= 0 || H % 64 != 0 || I % 64 != 0 ||
+      H > MAX_DIM || I > MAX_DIM)
+    return 0;
+  // status, the tile prefix [E+1], h [R, I]
+  return align_up(sizeof(DevStatus)) + align_up((size_t)(E + 1) * 4) + align_up((size_t)R * I * 2);
+}
+
+int32_t moe_expert_rows(const void* xr, const int32_t* offsets, int32_t R, int32_t E, int32_t H,
+                        int32_t I, const void* w13, const void* w2, const float* row_w,
+                        const int32_t* row_dest, void* y, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  if (R < 0 || E <= 0 || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+  if (E > MAX_E || H % 64 != 0 || I % 64 != 0 || H > MAX_DIM || I > MAX_DIM)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (R == 0) return MOE_OK;
+  if (!xr || !offsets || !w13 || !w2 || !row_dest || !y || y == xr) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_expert_rows_workspace_bytes(R, H, E, I);
+  if (!ws_ok(workspace, workspace_bytes, need)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = at<int>(workspace, 0);
+  int* tiles = at<int>(workspace, align_up(sizeof(DevStatus)));
+  __nv_bfloat16* h =
+      at<__nv_bfloat16>(workspace, align_up(sizeof(DevStatus)) + align_up((size_t)(E + 1) * 4));
+  RMOE_TRY(launch_status_reset(status, s));
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.status = status;
+  a.timeout_ns = DEFAULT_TIMEOUT_NS;
+  a.alt_group = -1;
+  a.row_start = offsets;
+  a.num_groups = E;
+  GemmArgs up = a, down = a;
+  up.k_steps = H / 64;
+  up.b_second = I;
+  up.out = h;
+  up.ldo = I;
+  up.n_valid = I;
+  down.k_steps = I / 64;
+  down.out = static_cast<__nv_bfloat16*>(y);
+  down.ldo = H;
+  down.n_valid = H;
+  down.row_scale = row_w;
+  down.dest_pos = row_dest;
+  const int sms = num_sms();
+  CUtensorMap tm_w13, tm_w2, tm_x, tm_h;
+  RMOE_TRY(make_tmap_3d(&tm_w13, w13, E, 2 * (uint64_t)I, H));
+  RMOE_TRY(make_tmap_3d(&tm_w2, w2, E, H, I));
+  if ((int64_t)R <= 64LL * E) {  // few rows per expert: swapped operands
+    const int chunk = (int64_t)R <= 20LL * E ? 32 : 128;
+    RMOE_TRY(make_tmap_2d_box(&tm_x, xr, R, H, 32));
+    RMOE_TRY(make_tmap_2d_box(&tm_h, h, R, I, 32));
+    const long long chunk_bound = R / chunk + E + 1;
+    up.n_tiles = (I + 127) / 128;
+    up.n_out_tile = 128;
+    down.n_tiles = (H + 127) / 128;
+    down.n_out_tile = 128;
+    RMOE_TRY(launch_grouped_gemm_swap(EPI_SWIGLU, chunk, tm_w13, tm_x, tm_w13, tm_x, up,
+                                      (int)std::min<long long>(sms, chunk_bound * up.n_tiles), s));
+    RMOE_TRY(launch_grouped_gemm_swap(EPI_ROWSCALE, chunk, tm_w2, tm_h, tm_w2, tm_h, down,
+                                      (int)std::min<long long>(sms, chunk_bound * down.n_tiles),
+                                      s));
+  } else {  // 256-row tiles on CTA pairs; the tile schedule from the row offsets
+    RMOE_TRY(make_tmap_2d(&tm_x, xr, R, H));
+    RMOE_TRY(make_tmap_2d(&tm_h, h, R, I));
+    RMOE_TRY(launch_tile_prefix(offsets, E, tiles, s));
+    up.mtile_start = tiles;
+    down.mtile_start = tiles;
+    const long long mt_bound = R / MTILE + E;
+    up.n_tiles = (I + 127) / 128;
+    up.n_out_tile = 128;
+    down.n_tiles = (H + 255) / 256;
+    down.n_out_tile = 256;
+    down.b_second = 128;
+    RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_x, tm_w13, tm_x, tm_w13, up,
+                                 (int)std::min<long long>(sms, 2LL * mt_bound * up.n_tiles), s));
+    RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, tm_h, tm_w2, down,
+                                 (int)std::min<long long>(sms, 2LL * mt_bound * down.n_tiles), s));
+  }
+  return MOE_OK;
+}
+
+int32_t moe_combine_rows(const void* y, const int32_t* row_of, int32_t T, int32_t H,
+                         int32_t top_k, const void* shared, const void* residual, void* out,
+                         void* stream) {
+  if (T < 0 || H <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (H % 64 != 0 || H > MAX_DIM || top_k > MAX_TOPK) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!y || !row_of || !out || out == y) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_combine_rows(y, row_of, top_k, T, H, shared, residual, out,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 int32_t moe_rmsnorm(const void* x, const float* gamma, float eps, int32_t T, int32_t H, void* xn,
                     void* stream) {
   if (T < 0 || H <= 0 || H % 64 != 0 || H > MAX_DIM || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;

@@ -147,6 +147,18 @@ cudaError_t launch_grouped_gemm_swap_fp8(int epi, int chunk, const CUtensorMap& 
 
 int num_sms();
 
+// ------------------------------------------------------------------ expert parallelism
+// ids[r] = the expert whose rows [offsets[e], offsets[e+1]) hold row r + offsets[0].
+cudaError_t launch_rows_expert_ids(const int* offsets, int E, int R, int* ids,
+                                   cudaStream_t stream);
+// tiles[g] = sum over g' < g of ceil((offsets[g'+1] - offsets[g']) / MTILE), g <= groups.
+cudaError_t launch_tile_prefix(const int* offsets, int groups, int* tiles, cudaStream_t stream);
+// out[t] = bf16( sum_{j<top_k} y[row_of[t*top_k+j]] (0 when < 0) [+ shared[t]] [+ residual[t]] ),
+// fp32 in that order.
+cudaError_t launch_combine_rows(const void* y, const int* row_of, int top_k, int T, int H,
+                                const void* shared, const void* residual, void* out,
+                                cudaStream_t stream);
+
 // ------------------------------------------------------------------ misc
 cudaError_t launch_rmsnorm(const void* x, const float* gamma, float eps, int T, int H, void* xn,
                            cudaStream_t stream);

@@ -102,6 +102,10 @@ def lib() -> ctypes.CDLL:
                                    vp, vp, cfgp, vp, sz, vp, vp, vp]),
         "moe_dense_ffn_workspace_bytes": (sz, [i32, i32, i32]),
         "moe_dense_ffn": (i32, [vp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
+        "moe_rows_expert_ids": (i32, [vp, i32, i32, vp, vp]),
+        "moe_expert_rows_workspace_bytes": (sz, [i32, i32, i32, i32]),
+        "moe_expert_rows": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "moe_combine_rows": (i32, [vp, vp, i32, i32, i32, vp, vp, vp, vp]),
         "moe_rmsnorm": (i32, [vp, vp, ctypes.c_float, i32, i32, vp, vp]),
         "moe_read_device_status": (i32, [vp, ctypes.POINTER(i32), vp]),
         "moe_selftest_wait_timeout": (i32, [vp, i64, vp]),
@@ -423,6 +427,70 @@ def dense_ffn(x: torch.Tensor, w13: torch.Tensor, w2: torch.Tensor,
         workspace = alloc_workspace(lib().moe_dense_ffn_workspace_bytes(T, H, I), x.device)
     _check(lib().moe_dense_ffn(_ptr(x), _ptr(w13), _ptr(w2), T, H, I, _ptr(residual), _ptr(out),
                                _ptr(workspace), workspace.numel(), _stream_ptr()), "moe_dense_ffn")
+    return out
+
+
+def rows_expert_ids(offsets: torch.Tensor, E: int) -> torch.Tensor:
+    """Expert id of every row of an expert-sorted row list (moe_rows_expert_ids):
+    int32 [offsets[E] - offsets[0]] from device offsets int32 [E+1]."""
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    R = int(offsets[E].item() - offsets[0].item())
+    ids = torch.empty(R, dtype=torch.int32, device=offsets.device)
+    _check(lib().moe_rows_expert_ids(_ptr(offsets), E, R, _ptr(ids), _stream_ptr()),
+           "moe_rows_expert_ids")
+    return ids
+
+
+def expert_rows(xr: torch.Tensor, offsets: torch.Tensor, w13: torch.Tensor, w2: torch.Tensor,
+                row_dest: torch.Tensor, row_w: Optional[torch.Tensor] = None,
+                y: Optional[torch.Tensor] = None, y_rows: Optional[int] = None,
+                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Routed experts on rows grouped by expert (moe_expert_rows):
+    y[row_dest[r]] = row_w[r] * SwiGLU_e(xr[r]) for r in [offsets[e], offsets[e+1]).
+    ``offsets`` may be a view into a longer offsets tensor (the local experts'
+    slice).  Returns y bf16 [y_rows (default R), H]."""
+    R, H = xr.shape
+    E = w13.shape[0]
+    I = w13.shape[1] // 2
+    _need(xr, "xr", torch.bfloat16, (R, H))
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _need(w13, "w13", torch.bfloat16, (E, 2 * I, H))
+    _need(w2, "w2", torch.bfloat16, (E, H, I))
+    _need(row_dest, "row_dest", torch.int32, (R,))
+    if row_w is not None:
+        _need(row_w, "row_w", torch.float32, (R,))
+    if y is None:
+        y = torch.empty((R if y_rows is None else y_rows, H), dtype=torch.bfloat16,
+                        device=xr.device)
+    elif y.dtype != torch.bfloat16 or y.dim() != 2 or y.shape[1] != H or not y.is_contiguous():
+        raise ValueError("y must be a contiguous bf16 [rows, H] tensor")
+    if workspace is None:
+        workspace = alloc_workspace(lib().moe_expert_rows_workspace_bytes(R, H, E, I), xr.device)
+    _check(lib().moe_expert_rows(_ptr(xr), _ptr(offsets), R, E, H, I, _ptr(w13), _ptr(w2),
+                                 _ptr(row_w), _ptr(row_dest), _ptr(y), _ptr(workspace),
+                                 workspace.numel(), _stream_ptr()), "moe_expert_rows")
+    return y
+
+
+def combine_rows(y: torch.Tensor, row_of: torch.Tensor, top_k: int,
+                 shared: Optional[torch.Tensor] = None, residual: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The restore through row_of (moe_combine_rows): out[t] = bf16(sum_j y[row_of[t, j]]
+    + shared[t] + residual[t]) in fp32, slot order, one rounding."""
+    H = y.shape[1]
+    T = row_of.numel() // top_k
+    if y.dtype != torch.bfloat16 or y.dim() != 2 or not y.is_cuda or not y.is_contiguous():
+        raise ValueError("y must be a contiguous CUDA bf16 [rows, H] tensor")
+    _need(row_of, "row_of", torch.int32, (T * top_k,))
+    for name, t in (("shared", shared), ("residual", residual)):
+        if t is not None:
+            _need(t, name, torch.bfloat16, (T, H))
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=y.device)
+    else:
+        _need(out, "out", torch.bfloat16, (T, H))
+    _check(lib().moe_combine_rows(_ptr(y), _ptr(row_of), T, H, top_k, _ptr(shared),
+                                  _ptr(residual), _ptr(out), _stream_ptr()), "moe_combine_rows")
     return out
 
 

@@ -215,3 +215,34 @@ def test_forward_fp8_rejects_bad_arguments_on_the_host(L):
     assert call(cfg=BlockConfig(T=64, H=250).c()) == 2
     z = BlockConfig(T=0, H=256, I=128, I_shared=128).c()
     assert call(cfg=z, x=None, q=(None,) * 8, o=None, ws=None, nbytes=0) == 0
+
+
+def test_expert_parallel_entries_reject_bad_arguments_on_the_host(L):
+    # moe_rows_expert_ids
+    assert L.moe_rows_expert_ids(FAKE, 0, 10, FAKE, None) == 1
+    assert L.moe_rows_expert_ids(FAKE, 129, 10, FAKE, None) == 1
+    assert L.moe_rows_expert_ids(None, 8, 10, FAKE, None) == 1
+    assert L.moe_rows_expert_ids(None, 8, 0, None, None) == 0
+    # moe_expert_rows
+    need = L.moe_expert_rows_workspace_bytes(100, 256, 8, 128)
+    assert need >= 100 * 128 * 2
+    assert L.moe_expert_rows_workspace_bytes(100, 250, 8, 128) == 0
+    y = ctypes.c_void_p(0x20000)
+    args = lambda **k: [k.get("xr", FAKE), FAKE, k.get("R", 100), k.get("E", 8), k.get("H", 256),
+                        k.get("I", 128), FAKE, FAKE, None, k.get("dest", FAKE), k.get("y", y),
+                        k.get("ws", FAKE), k.get("nbytes", need), None]
+    assert L.moe_expert_rows(*args(xr=None)) == 1
+    assert L.moe_expert_rows(*args(dest=None)) == 1
+    assert L.moe_expert_rows(*args(y=FAKE)) == 1            # y aliases xr
+    assert L.moe_expert_rows(*args(E=129)) == 2
+    assert L.moe_expert_rows(*args(H=250)) == 2
+    assert L.moe_expert_rows(*args(nbytes=need - 1)) == 3
+    assert L.moe_expert_rows(*args(ws=ctypes.c_void_p(0x10010))) == 3
+    assert L.moe_expert_rows(*args(R=0, xr=None, y=None)) == 0
+    # moe_combine_rows
+    out = ctypes.c_void_p(0x30000)
+    assert L.moe_combine_rows(None, FAKE, 10, 256, 8, None, None, out, None) == 1
+    assert L.moe_combine_rows(FAKE, FAKE, 10, 256, 8, None, None, FAKE, None) == 1  # out is y
+    assert L.moe_combine_rows(FAKE, FAKE, 10, 250, 8, None, None, out, None) == 2
+    assert L.moe_combine_rows(FAKE, FAKE, 10, 256, 17, None, None, out, None) == 2
+    assert L.moe_combine_rows(None, None, 0, 256, 8, None, None, None, None) == 0
