@@ -192,12 +192,14 @@ def ep_forward(x: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor, w13_local:
         xr, ir, wr = p["xp"], row_ids, p["w_of"]
     R_in = int(sum(recv))
     # 3. this rank's experts on the received rows, results in received order
-    cfg1 = dataclasses.replace(cfg, T=R_in, top_k=1)
     if R_in > 0:
+        cfg1 = dataclasses.replace(cfg, T=R_in, top_k=1)
         q = be.permute(ir.reshape(R_in, 1), wr.reshape(R_in, 1), xr, cfg1)
-        local_offsets = q["expert_offsets"][base:base + el + 1]
-    yr = be.expert_rows(q["xp"], local_offsets, w13_local, w2_local, q["tok_of"], q["w_of"],
-                        R_in) if R_in > 0 else xr.new_empty((0, x.shape[1]))
+        local_offsets = q["expert_offsets"][base:base + el + 1]  # this rank's experts
+        yr = be.expert_rows(q["xp"], local_offsets, w13_local, w2_local, q["tok_of"],
+                            q["w_of"], R_in)
+    else:
+        yr = xr.new_empty((0, x.shape[1]))
     # 4. combine: the weighted rows back to their tokens' ranks, in the order sent
     yb = _all_to_all(yr, recv, send, group) if world > 1 else yr
     if T == 0:
