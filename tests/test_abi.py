@@ -246,3 +246,18 @@ def test_expert_parallel_entries_reject_bad_arguments_on_the_host(L):
     assert L.moe_combine_rows(FAKE, FAKE, 10, 250, 8, None, None, out, None) == 2
     assert L.moe_combine_rows(FAKE, FAKE, 10, 256, 17, None, None, out, None) == 2
     assert L.moe_combine_rows(None, None, 0, 256, 8, None, None, None, None) == 0
+
+
+def test_public_header_is_plain_c():
+    """include/*.h is a C ABI: it must compile as C99 (and as C++) with no torch types."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        for lang, std in (("c", "c99"), ("c++", "c++17")):
+            r = subprocess.run(["gcc", "-fsyntax-only", f"-std={std}", "-Wall", "-Werror", "-x",
+                                lang, h], capture_output=True, text=True)
+            assert r.returncode == 0, (h, lang, r.stderr)
+        src = open(h).read()
+        assert "#include <torch" not in src and "torch::" not in src and "at::" not in src
