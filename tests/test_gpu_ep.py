@@ -12,9 +12,7 @@ from routed_moe_layer_b200 import inputs, ops
 from routed_moe_layer_b200.dist import ep_forward
 from routed_moe_layer_b200.ops import BlockConfig
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skip(reason="the expert-parallel entry points have not been run on a "
-                                      "GPU yet")]
+pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
 
