@@ -110,6 +110,34 @@ def _block_index_transposed(codes, scale_exp, block=128):
     return om.fp8_e4m3_decode(codes) * scale[..., cols[None, :], rows[:, None]]
 
 
+def _rms_gamma_divided(x, eps=1e-6, gamma=None):
+    xd = x.astype(np.float64)
+    r = xd / np.sqrt(np.mean(xd * xd, axis=1, keepdims=True) + eps)
+    return r if gamma is None else r / gamma.astype(np.float64)[None, :]
+
+
+def _rms_gamma_reversed(x, eps=1e-6, gamma=None):
+    xd = x.astype(np.float64)
+    r = xd / np.sqrt(np.mean(xd * xd, axis=1, keepdims=True) + eps)
+    return r if gamma is None else r * gamma.astype(np.float64)[::-1][None, :]
+
+
+def _rms_eps_outside_root(x, eps=1e-6, gamma=None):
+    xd = x.astype(np.float64)
+    r = xd / (np.sqrt(np.mean(xd * xd, axis=1, keepdims=True)) + eps)
+    return r if gamma is None else r * gamma.astype(np.float64)[None, :]
+
+
+def _always_renormalise(s, ids, rsf, norm_topk_prob=True):
+    sel = np.take_along_axis(s.astype(np.float64), ids.astype(np.int64), axis=1)
+    return rsf * sel / sel.sum(axis=1, keepdims=True)
+
+
+def _never_renormalise(s, ids, rsf, norm_topk_prob=True):
+    sel = np.take_along_axis(s.astype(np.float64), ids.astype(np.int64), axis=1)
+    return rsf * sel
+
+
 PIN_TESTS = [
     lambda: pins.test_hand_worked_golden_example(),
     lambda: [pins.test_selection_matches_brute_force(*a) for a in
@@ -120,6 +148,9 @@ PIN_TESTS = [
     lambda: pins.test_single_expert_is_textbook_swiglu_plus_shared(),
     lambda: pins.test_swiglu_gate_up_order_and_w2_orientation(),
     lambda: pins.test_padding_mask_keeps_only_the_shared_expert(),
+    lambda: pins.test_hand_worked_golden_example_without_renormalisation(),
+    lambda: pins.test_rmsnorm_gamma_multiplies_each_channel(),
+    lambda: pins.test_rmsnorm_eps_inside_the_square_root(),
     lambda: fp8_pins.test_e4m3_decode_matches_torch_float8_on_every_code(),
     lambda: fp8_pins.test_ue8m0_scales(),
     lambda: fp8_pins.test_block_scales_land_on_their_blocks_ragged_non_square(),
@@ -139,6 +170,16 @@ MUTATIONS = {
     "w2_misoriented": [(om, "swiglu_mlp", _w2_transposed_use),
                        (pins, "swiglu_mlp", _w2_transposed_use)],
     "shared_expert_scaled": [(pins, "moe_forward", _scaled_shared)],
+    "rmsnorm_gamma_divided": [(om, "rmsnorm", _rms_gamma_divided),
+                              (pins, "rmsnorm", _rms_gamma_divided)],
+    "rmsnorm_gamma_wrong_channel": [(om, "rmsnorm", _rms_gamma_reversed),
+                                    (pins, "rmsnorm", _rms_gamma_reversed)],
+    "rmsnorm_eps_outside_root": [(om, "rmsnorm", _rms_eps_outside_root),
+                                 (pins, "rmsnorm", _rms_eps_outside_root)],
+    "norm_topk_prob_ignored": [(om, "routing_weights", _always_renormalise),
+                               (pins, "routing_weights", _always_renormalise)],
+    "renormalisation_dropped": [(om, "routing_weights", _never_renormalise),
+                                (pins, "routing_weights", _never_renormalise)],
     "padding_mask_ignored": [(om, "apply_token_mask", _mask_ignored)],
     "padding_drops_shared_expert": [(pins, "moe_forward", _forward_mask_kills_shared)],
     "e4m3_exponent_bias_8": [(om, "fp8_e4m3_decode", _e4m3_bias_8),

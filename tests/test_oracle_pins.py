@@ -189,6 +189,21 @@ def test_hand_worked_golden_example():
     assert np.all(margin > 0.09)
 
 
+def test_hand_worked_golden_example_without_renormalisation():
+    """norm_topk_prob off: the same experts, each weighted by 2.5 times its raw
+    score (hand-worked values in the golden file)."""
+    g, x, Wr, bias, w13, w2, ws13, ws2, cfg = _golden_inputs()
+    cfg = MoeConfig(E=8, I=1, I_shared=1, top_k=2, n_group=4, topk_group=2,
+                    norm_topk_prob=False)
+    out, ids, w, _ = moe_forward(x, Wr, bias, w13, w2, ws13, ws2, cfg)
+    assert ids.tolist() == g["expected_ids"]
+    np.testing.assert_allclose(w, g["expected_weights_no_renorm"], rtol=1e-6)
+    np.testing.assert_allclose(out, g["expected_out_no_renorm"], rtol=1e-6)
+    ids_r, w_r, _, _ = route(x, Wr, bias, cfg)
+    assert ids_r.tolist() == g["expected_ids"]
+    np.testing.assert_allclose(w_r, g["expected_weights_no_renorm"], rtol=1e-6)
+
+
 # ----------------------------------------------------------------------------
 # Expert math: closed forms and special cases
 # ----------------------------------------------------------------------------
@@ -338,6 +353,37 @@ def test_rmsnorm_unit_rms_and_bf16_rounding():
     np.testing.assert_array_equal(bf16_round(vals), exp)
     t = torch.from_numpy(rng.standard_normal(4096).astype(np.float32))
     np.testing.assert_array_equal(bf16_round(t.numpy()), t.to(torch.bfloat16).float().numpy())
+
+
+def test_rmsnorm_gamma_multiplies_each_channel():
+    """Rows whose mean square is a perfect square, with eps = 0, and a gamma of
+    distinct powers of two: every output is a short binary fraction written out
+    by hand.  A gamma divided instead of multiplied, or read at the wrong
+    channel, changes them."""
+    x = np.array([[3.0, -3.0, 3.0, -3.0],     # mean square 9 -> x / 3
+                  [0.0, 4.0, 0.0, 0.0],       # mean square 4 -> x / 2
+                  [1.0, 1.0, 1.0, 1.0]])      # mean square 1 -> x
+    gamma = np.array([2.0, 0.5, 4.0, 0.25])
+    exp = np.array([[2.0, -0.5, 4.0, -0.25],
+                    [0.0, 1.0, 0.0, 0.0],
+                    [2.0, 0.5, 4.0, 0.25]])
+    np.testing.assert_array_equal(rmsnorm(x, eps=0.0, gamma=gamma), exp)
+    # no gamma is gamma = 1
+    np.testing.assert_array_equal(rmsnorm(x, eps=0.0), exp / gamma[None, :])
+
+
+def test_rmsnorm_eps_inside_the_square_root():
+    """A constant row a with a^2 = eps: a / sqrt(a^2 + eps) = 1 / sqrt(2)
+    exactly in real arithmetic.  eps outside the root would give
+    a / (|a| + eps) (~0.999), a dropped eps 1."""
+    a, eps = 1e-3, 1e-6
+    x = np.full((2, 64), a)
+    x[1] = -a
+    r = rmsnorm(x, eps=eps)
+    np.testing.assert_allclose(r[0], 1.0 / math.sqrt(2.0), rtol=1e-12)
+    np.testing.assert_allclose(r[1], -1.0 / math.sqrt(2.0), rtol=1e-12)
+    # eps only matters relative to the mean square: a large row is unaffected
+    np.testing.assert_allclose(rmsnorm(np.full((1, 64), 1e3), eps=eps), 1.0, rtol=1e-12)
 
 
 def test_invalid_configs_raise():
