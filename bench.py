@@ -41,7 +41,11 @@ from routed_moe_layer_b200.ops import BlockConfig  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and TFLOP/s at T~19.4k bf16; % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 10  # router 3, permute 3 + gather, expert up/down (+shared), combine
+def kernels_per_step(T: int) -> int:
+    """Launches of one block forward: router 3 (Wr split, GEMM, selection), permutation
+    3 (one kernel up to 1024 tokens), gather, expert up, expert down (the shared expert
+    folded into both), combine."""
+    return 3 + (1 if T <= 1024 else 3) + 1 + 2 + 1
 
 
 def flops_per_token(cfg: BlockConfig) -> float:
@@ -49,11 +53,29 @@ def flops_per_token(cfg: BlockConfig) -> float:
     return (2.0 * cfg.E * cfg.H + cfg.top_k * 6.0 * cfg.H * cfg.I + 6.0 * cfg.H * cfg.I_shared)
 
 
-def algorithmic_bytes(cfg: BlockConfig, experts_used: int) -> float:
-    """Weights of the experts that receive a token + shared + router + x in + out."""
-    per_expert = 3.0 * cfg.I * cfg.H * 2
-    return (experts_used * per_expert + 3.0 * cfg.I_shared * cfg.H * 2 + cfg.E * cfg.H * 4 +
+DATASHEET_HBM_GBS = 8000.0  # B200 HBM3e, nominal
+
+
+def weight_bytes_per_element(fp8: bool) -> float:
+    """bf16: 2 bytes; FP8: one E4M3 byte plus one scale byte per 128 x 128 block."""
+    return 1.0 + 1.0 / (128 * 128) if fp8 else 2.0
+
+
+def algorithmic_bytes(cfg: BlockConfig, experts_used: int, fp8: bool = False) -> float:
+    """Weights of the experts that receive a token + shared + router + x in + out
+    (no implementation intermediates: gathered rows, h and expert outputs are not counted)."""
+    b = weight_bytes_per_element(fp8)
+    per_expert = 3.0 * cfg.I * cfg.H * b
+    return (experts_used * per_expert + 3.0 * cfg.I_shared * cfg.H * b + cfg.E * cfg.H * 4 +
             cfg.E * 4 + 2.0 * cfg.T * cfg.H * 2)
+
+
+def up_launch_bytes(cfg: BlockConfig, experts_used: int, fp8: bool = False) -> float:
+    """The expert-up launch's share of the algorithmic bytes: w13 of the used
+    experts, ws13 and the tokens x once (no intermediates)."""
+    b = weight_bytes_per_element(fp8)
+    return (experts_used * 2.0 * cfg.I * cfg.H * b + 2.0 * cfg.I_shared * cfg.H * b +
+            cfg.T * cfg.H * 2.0)
 
 
 class CallTimer:
@@ -278,6 +300,9 @@ def run_ours(args, world, rank, local):
     # weights: identical on every rank; tokens: a different batch per rank
     gen_dev = dev if layers > 1 else "cpu"
     dense = wl.dense_I > 0  # a dense feed-forward layer instead of the MoE block
+    fp8 = bool(args.fp8)
+    if fp8 and (dense or layers > 1):
+        raise SystemExit("--fp8 applies to the single-layer MoE workloads")
     weights = []
     for l in range(layers):
         if dense:
@@ -285,6 +310,9 @@ def run_ours(args, world, rank, local):
         else:
             wd = inputs.make_weights(wl.H, wl.seed, device=gen_dev, layer=l,
                                      hot_experts=wl.hot_experts, hot_bias=wl.hot_bias)
+        if fp8:  # E4M3 expert weights from the same normal draws, router unchanged
+            wd = dict(Wr=wd["Wr"], bias=wd["bias"],
+                      **inputs.make_fp8_weights(wl.H, wl.seed, device=dev, layer=l))
         weights.append({k: (None if v is None else v.to(dev)) for k, v in wd.items()})
     x_host = inputs.make_tokens(wl.T, wl.H, rank_token_seed(wl.seed, rank)).pin_memory()
     x = x_host.to(dev)
@@ -305,6 +333,10 @@ def run_ours(args, world, rank, local):
             if timer is not None:
                 timer.end.record(torch.cuda.current_stream())
             return out
+        if fp8:
+            w = weights[0]
+            return ops.forward_fp8(xin, w["Wr"], w["bias"], w, cfg, out=out, workspace=ws,
+                                   timer=timer, topk_ids=ids, token_mask=mask_dev)
         if layers == 1:
             w = weights[0]
             return ops.forward(xin, w["Wr"], w["bias"], w["w13"], w["w2"], w["ws13"], w["ws2"],
@@ -388,7 +420,7 @@ def run_ours(args, world, rank, local):
     _barrier(world)
     e2e_serial_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     e2e_ms, e2e_mode = e2e_serial_ms, "serial: copy in, block, copy out, one batch at a time"
-    if layers == 1 and mask_dev is None and not dense:
+    if layers == 1 and mask_dev is None and not dense and not fp8:
         # the library's host-batch entry point: every step's batch is copied in
         # and its output copied out, the copies of the neighbouring batches
         # overlapping each batch's kernels (two copy streams)
@@ -442,7 +474,7 @@ def run_ours(args, world, rank, local):
         peak_tf = peaks.get(peak_key, peaks["bf16_tflops"])
         achieved = up_flops / (up_ms * 1e-3) / 1e12
         layer_ms = ms / layers
-        hbm_bytes = (algorithmic_bytes(cfg, experts_used) if not dense else
+        hbm_bytes = (algorithmic_bytes(cfg, experts_used, fp8) if not dense else
                      3.0 * wl.dense_I * wl.H * 2 + 2.0 * wl.T * wl.H * 2)
         t_flop = flops_per_step / peak_tf / 1e12
         t_hbm = hbm_bytes / peaks["hbm_gbs"] / 1e9
@@ -450,18 +482,22 @@ def run_ours(args, world, rank, local):
         kernel = ("grouped_gemm_swap_kernel<SwiGLU> (expert up, shared expert folded in)"
                   if swapped else
                   "grouped_gemm_kernel<SwiGLU> (expert up, shared expert folded in)")
+        if fp8:
+            swapped = True  # FP8 weights: the dequantising swapped kernel at every size
+            kernel = "grouped_gemm_swap_fp8_kernel<SwiGLU> (expert up, E4M3 weights, shared folded in)"
         if dense:
             swapped = wl.T <= 64
             kernel = "grouped_gemm_kernel<SwiGLU> + <RowScale> (dense layer: both GEMMs)"
         if t_hbm > t_flop:
-            # HBM-bound layer: the expert-up launch streams w13 of the used experts and
-            # ws13, reads the gathered rows and x, writes h
-            up_bytes = (experts_used * 2.0 * cfg.I * cfg.H * 2 + 2.0 * cfg.I_shared * cfg.H * 2 +
-                        up_rows * cfg.H * 2 + up_rows * cfg.I * 2)
+            # HBM-bound layer: the expert-up launch's algorithmic bytes are w13 of the
+            # used experts, ws13 and the tokens once (the gathered rows it reads and
+            # the h it writes are intermediates and are not counted)
+            up_bytes = up_launch_bytes(cfg, experts_used, fp8)
             ach = up_bytes / (up_ms * 1e-3) / 1e9
             rf = {"bound": "hbm", "kernel": kernel, "achieved": ach, "peak": peaks["hbm_gbs"],
                   "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
                   "peak_source": f"{peak_src} HBM copy bandwidth",
+                  "frac_of_datasheet_8000_gbs": ach / DATASHEET_HBM_GBS,
                   "algorithmic_bytes_per_launch": up_bytes, "flops_per_launch": up_flops}
         else:
             rf = {"bound": "tensor", "kernel": kernel,
@@ -472,6 +508,9 @@ def run_ours(args, world, rank, local):
                          measured_traffic("grouped_gemm_kernel<EPI_SWIGLU>", wl.name))
         rf["traffic_unit"] = "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
         rf["layer_roofline_frac"] = max(t_flop, t_hbm) / (layer_ms * 1e-3)
+        if t_hbm > t_flop:
+            rf["layer_hbm_frac_of_datasheet_8000_gbs"] = (
+                hbm_bytes / (DATASHEET_HBM_GBS * 1e9) / (layer_ms * 1e-3))
         cpu_tps, cores, sample = (None, None, None)
         if world == 1 and not args.no_cpu_baseline:
             cpu_tps, cores, sample = cpu_oracle_sample(args.config, target_s=args.cpu_seconds)
@@ -486,6 +525,8 @@ def run_ours(args, world, rank, local):
                        "tokens_per_gpu_per_step": tok_per_step,
                        "padding_tokens_per_layer": n_pad,
                        "dense_intermediate": wl.dense_I or None,
+                       "expert_weights": ("fp8 e4m3, one power-of-two scale per 128x128 block"
+                                          if fp8 else "bf16"),
                        "l2": ("inputs larger than L2: " +
                               ("the layer's 85 MB of weights, 80 MB of tokens in and out"
                                if dense else "1.2 GB of expert weights read per layer"))},
@@ -503,7 +544,7 @@ def run_ours(args, world, rank, local):
                     "d2h_bytes_per_step": int(out_host.numel() * 2),
                     "mode": e2e_mode,
                     "serial_value": total_tokens / (e2e_serial_ms * 1e-3)},
-            "gpu_launches": ((2 if dense else KERNELS_PER_STEP + (1 if layers > 1 else 0)) *
+            "gpu_launches": ((2 if dense else kernels_per_step(wl.T) + (1 if layers > 1 else 0)) *
                              layers * args.steps),
             "clocks": sampler.summary(),
         }
@@ -525,6 +566,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=64,
                     help="tokens per step for --impl reference (bounded CPU sample)")
     ap.add_argument("--ref-warmup", action="store_true")
+    ap.add_argument("--fp8", action="store_true",
+                    help="FP8 (E4M3, block-scaled) expert weights (single-layer MoE workloads)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")

@@ -178,7 +178,9 @@ MOE_API int32_t moe_permute(const int32_t* topk_ids, const float* topk_w, const 
  *   launches nothing.  The call allocates nothing (no cudaMalloc/cudaFree).
  *   The first call on a device looks up the array's device address (once
  *   per device, with that device current); make that first call before any
- *   stream capture.
+ *   stream capture.  A device reset (cudaDeviceReset) frees the array with
+ *   the device's context; the next call sees a new context and looks the
+ *   address up again, so it also belongs before any capture.
  *   Every call on a device shares the one array and it keeps the last call's
  *   contents: calls that overlap on the GPU (different streams, no ordering)
  *   race and give wrong results.  An expert id outside [0,E) is skipped and

@@ -406,8 +406,9 @@ template <int EPI>
 cudaError_t launch_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
                        const CUtensorMap& tmB2, const GemmArgs& args, int grid,
                        cudaStream_t stream) {
-  static cudaError_t attr = cudaFuncSetAttribute(
-      grouped_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  static std::atomic<int> smem_set[MAX_DEVICES];
+  const cudaError_t attr =
+      set_smem_limit_per_device(grouped_gemm_kernel<EPI>, (int)SMEM_BYTES, smem_set);
   if (attr != cudaSuccess) return attr;
   grid &= ~1;  // clusters of two CTAs
   if (grid < 2) grid = 2;

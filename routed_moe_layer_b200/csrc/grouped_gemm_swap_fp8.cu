@@ -583,9 +583,9 @@ cudaError_t launch_swap8(const CUtensorMap& tmW, const CUtensorMap& tmX, const C
                          int grid, cudaStream_t stream) {
   constexpr size_t smem = smem_bytes8<EPI, CHUNK>();
   static_assert(smem <= 227 * 1024, "shared memory");
-  static cudaError_t attr =
-      cudaFuncSetAttribute(grouped_gemm_swap_fp8_kernel<EPI, CHUNK>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static std::atomic<int> smem_set[MAX_DEVICES];
+  const cudaError_t attr =
+      set_smem_limit_per_device(grouped_gemm_swap_fp8_kernel<EPI, CHUNK>, (int)smem, smem_set);
   if (attr != cudaSuccess) return attr;
   if (grid < 1) grid = 1;
   return launch_chained(grouped_gemm_swap_fp8_kernel<EPI, CHUNK>, dim3(grid), dim3(THREADS), smem,

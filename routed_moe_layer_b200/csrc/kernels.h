@@ -5,9 +5,26 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 namespace rmoe {
+
+// A kernel's dynamic shared-memory limit is an attribute of the kernel in one
+// device's context, so it is set once per device: `done` is a per-call-site
+// table indexed by device ordinal (devices beyond it set it on every launch).
+constexpr int MAX_DEVICES = 64;
+template <typename... KArgs>
+cudaError_t set_smem_limit_per_device(void (*k)(KArgs...), int bytes,
+                                      std::atomic<int> (&done)[MAX_DEVICES]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < MAX_DEVICES && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < MAX_DEVICES) done[dev].store(1, std::memory_order_release);
+  return e;
+}
 
 // Launches kernel k chained to the previous work of the stream (programmatic
 // stream serialisation; the kernel itself waits with pdl_wait before reading

@@ -578,8 +578,8 @@ cudaError_t launch_router(const void* x, const float* Wr, const float* bias, con
   if (err != cudaSuccess) return err;
   err = make_tmap_3d_box(&tmW3, Wr3, 3, (uint64_t)E, (uint64_t)H, (uint32_t)NP);
   if (err != cudaSuccess) return err;
-  err = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)R_SMEM_BYTES);
+  static std::atomic<int> smem_set[MAX_DEVICES];
+  err = set_smem_limit_per_device(router_gemm_kernel, (int)R_SMEM_BYTES, smem_set);
   if (err != cudaSuccess) return err;
   const int items = tiles * (RBN / NP);
   const int grid = items < num_sms() ? items : num_sms();

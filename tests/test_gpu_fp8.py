@@ -18,8 +18,7 @@ from routed_moe_layer_b200 import inputs, ops
 from routed_moe_layer_b200.ops import BlockConfig
 from tests import parity
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skip(reason="the FP8 kernel has not been run on a GPU yet")]
+pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
 

@@ -102,6 +102,34 @@ def test_router_bias_forces_selection_not_weights():
         assert torch.equal(w[t][o], w0[t][o0])
 
 
+@pytest.mark.parametrize("T,H,I", [(1, 256, 128), (300, 512, 256), (2048, 1024, 768),
+                                   (5000, 256, 128)])
+def test_routing_without_renormalisation(T, H, I):
+    """norm_topk_prob off: weights are rsf x the raw scores of the chosen
+    experts (no renormalisation); the router (one warp per token up to 4096
+    tokens, half warps above) and the whole block (swapped and tiled GEMMs)
+    against the oracle with the same option.  rsf = 0.3 keeps the weights'
+    sum near 2 (eight sigmoids of about 0.85): with 2.5 it would be about 17,
+    routed outputs some 7x those of the renormalised block, and the
+    tolerance's absolute floor (2e-2) would no longer match the outputs' scale."""
+    cfg = BlockConfig(T=T, H=H, I=I, I_shared=I, norm_topk_prob=False,
+                      routed_scaling_factor=0.3)
+    d = inputs.make_block_inputs(T, H, seed=31 + T, I=I, I_shared=I, unit_scale=True)
+    dd = _dev(d)
+    dn = parity.np_inputs(d)
+    ids_r, w_r = ops.route(dd["x"], dd["Wr"], dd["bias"], cfg)
+    torch.cuda.synchronize()
+    parity.check_routing(ids_r, w_r, dn["x"], dn["Wr"], dn["bias"], cfg)
+    # not renormalised: the sums are rsf x (sum of 8 sigmoids), not rsf
+    assert not np.allclose(w_r.sum(1).cpu().numpy(), 0.3, rtol=1e-3)
+    if T > 2048:
+        return
+    out, ids, w = _run(dd, cfg)
+    assert torch.equal(ids, ids_r) and torch.equal(w, w_r)
+    rep = parity.check_output(out, ids, dn, cfg)
+    assert rep["rms_rel"] < 1e-2, rep
+
+
 # ------------------------------------------------------------------ permutation
 # T <= 1024 runs the single-CTA path, larger T the three-kernel path
 @pytest.mark.parametrize("T,E,k", [(1, 8, 2), (255, 128, 8), (256, 128, 8), (257, 128, 8),

@@ -54,10 +54,12 @@ def _noalloc(ids, w, x, cfg):
     return dict(expert_offsets=offsets, row_of=row_of, tok_of=tok_of, w_of=w_of, xp=xp)
 
 
-def test_noalloc_permute_matches_workspace_permute_twice():
+def test_noalloc_permute_matches_workspace_permute_on_consecutive_calls():
     # the second call has fewer tokens and another expert count, so stale
-    # histogram rows of the first call would show up if they were read
-    for T, E, k, seed in ((5000, 128, 8, 1), (1234, 64, 6, 2)):
+    # histogram rows of the first call would show up if they were read; the
+    # third (T <= 1024) runs the one-CTA path, which writes the tile prefix
+    # and the status word into the same array after the larger calls
+    for T, E, k, seed in ((5000, 128, 8, 1), (1234, 64, 6, 2), (240, 128, 8, 3)):
         cfg = BlockConfig(T=T, H=256, E=E, top_k=k, n_group=1, topk_group=1)
         ids, w, x = _inputs(T, E, k, cfg.H, seed)
         got = _noalloc(ids, w, x, cfg)
