@@ -337,14 +337,16 @@ MOE_API int32_t moe_expert_rows(const void* xr, const int32_t* offsets, int32_t 
 
 /* The restore with each token's routed rows addressed through row_of:
  *   out[t] = bf16( sum_{j<top_k} y[row_of[t*top_k+j]] [+ shared[t]] [+ residual[t]] )
- * summed in fp32 in that order (a row_of entry < 0 adds 0), rounded once -- the
- * order and rounding of moe_forward's restore ([S2] "_restore_tokens").
- *   y device bf16 [rows,H]; row_of device int32 [T,top_k]; shared, residual
+ * summed in fp32 in that order, rounded once -- the order and rounding of
+ * moe_forward's restore ([S2] "_restore_tokens").  A row_of entry outside
+ * [0, R) adds 0, like a rejected expert id (there is no status word here: such
+ * an entry is not reported).
+ *   y device bf16 [R,H]; row_of device int32 [T,top_k]; shared, residual
  *   device bf16 [T,H] or NULL; out device bf16 [T,H] (may be residual).
- * H a multiple of 64 (<= 16384); top_k in 1..16. */
-MOE_API int32_t moe_combine_rows(const void* y, const int32_t* row_of, int32_t T, int32_t H,
-                                 int32_t top_k, const void* shared, const void* residual,
-                                 void* out, void* stream);
+ * H a multiple of 64 (<= 16384); top_k in 1..16; R >= 0. */
+MOE_API int32_t moe_combine_rows(const void* y, int32_t R, const int32_t* row_of, int32_t T,
+                                 int32_t H, int32_t top_k, const void* shared,
+                                 const void* residual, void* out, void* stream);
 
 /* RMSNorm with fp32 accumulation ([S2]: RMSNorm accumulates in fp32), for a
  * residual stack of blocks: xn = bf16(x * rsqrt(mean(x^2) + eps) * gamma).

@@ -143,6 +143,42 @@ RouterParams router_params(const moe_cfg_t& c) {
     if (e_ != cudaSuccess) return MOE_ERR_CUDA; \
   } while (0)
 
+// A group's last tile with at most this many rows runs with swapped operands
+// inside the pair kernel (TailMaps): it then costs about its rows rounded to
+// 16 instead of a full 256-row tile, with the same bits.
+constexpr int TAIL_MAX_ROWS = 192;
+
+// The maps of the swapped last tiles of one pair-kernel launch.
+// SwiGLU: A rows (a, a2) in 32-row boxes, weights (w, w2) in 64-row boxes.
+cudaError_t tail_maps_swiglu(TailMaps* t, const void* a, uint64_t a_rows, const void* a2,
+                             uint64_t a2_rows, uint64_t K, const void* w, uint64_t groups,
+                             uint64_t w_rows, const void* w2, uint64_t w2_rows) {
+  cudaError_t e;
+  if ((e = make_tmap_2d_box(&t->x, a, a_rows, K, 32)) != cudaSuccess) return e;
+  if ((e = make_tmap_2d_box(&t->x2, a2 ? a2 : a, a2 ? a2_rows : a_rows, K, 32)) != cudaSuccess)
+    return e;
+  if ((e = make_tmap_3d_box(&t->w, w, groups, w_rows, K, 64)) != cudaSuccess) return e;
+  if ((e = make_tmap_3d_box(&t->w2, w2 ? w2 : w, w2 ? 1 : groups, w2 ? w2_rows : w_rows, K, 64)) !=
+      cudaSuccess)
+    return e;
+  t->max_rows = TAIL_MAX_ROWS;
+  return cudaSuccess;
+}
+
+// Weighted down projection: A rows (a, a2) in 32-row boxes, the regular weight maps.
+cudaError_t tail_maps_rowscale(TailMaps* t, const void* a, uint64_t a_rows, const void* a2,
+                               uint64_t a2_rows, uint64_t K, const CUtensorMap& w,
+                               const CUtensorMap& w2) {
+  cudaError_t e;
+  if ((e = make_tmap_2d_box(&t->x, a, a_rows, K, 32)) != cudaSuccess) return e;
+  if ((e = make_tmap_2d_box(&t->x2, a2 ? a2 : a, a2 ? a2_rows : a_rows, K, 32)) != cudaSuccess)
+    return e;
+  t->w = w;
+  t->w2 = w2;
+  t->max_rows = TAIL_MAX_ROWS;
+  return cudaSuccess;
+}
+
 // Host checks of moe_forward (the configuration already checked).
 int32_t check_forward_args(const moe_cfg_t& c, const void* x, const float* Wr, const float* bias,
                            const void* w13, const void* w2, const void* ws13, const void* ws2,
@@ -340,6 +376,7 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
   o.xp = xp;
   o.mask = rp.mask;
   RMOE_TRY(launch_permute(ids, tw, x, c.T, c.H, c.E, c.top_k, o, s));
+  const void* residual = opts ? opts->residual : nullptr;
 
   // tiles of MTILE rows, each computed by a pair of CTAs; every group adds at
   // most one partial tile
@@ -373,7 +410,11 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
       g.ldo = c.I;
       g.n_valid = c.I;
       const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
-      RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_xp, tm_w13, tm_x, tm_ws13, g, grid, s));
+      TailMaps tails;
+      RMOE_TRY(tail_maps_swiglu(&tails, xp, R, fused ? x : nullptr, T, c.H, w13, c.E,
+                                2 * (uint64_t)c.I, fused ? ws13 : nullptr,
+                                2 * (uint64_t)c.I_shared));
+      RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_xp, tm_w13, tm_x, tm_ws13, g, grid, s, &tails));
     }
     RMOE_TRY(record(MOE_STAGE_EXPERT_DOWN));
     {  // Y[t*slots + j] = w_tj * (h . W2^T) per expert; shared rows to slot top_k, unscaled
@@ -397,7 +438,10 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
       g.dest_mul = slots;
       g.dest_add = c.top_k;
       const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
-      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, tm_h, tm_ws2, g, grid, s));
+      TailMaps tails;
+      RMOE_TRY(tail_maps_rowscale(&tails, h, h_rows, nullptr, 0, c.I, tm_w2,
+                                  fused ? tm_ws2 : tm_w2));
+      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, tm_h, tm_ws2, g, grid, s, &tails));
     }
     RMOE_TRY(record(MOE_STAGE_SHARED_EXPERT));
     if (c.I_shared > 0 && !fused) {
@@ -434,7 +478,6 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
     }
   }
   RMOE_TRY(record(MOE_STAGE_COMBINE));
-  const void* residual = opts ? opts->residual : nullptr;
   RMOE_TRY(launch_combine_slots(Y, row_of, c.top_k, c.T, c.H, slots, residual, out, s));
   RMOE_TRY(record(MOE_NUM_STAGES));
   return MOE_OK;
@@ -987,14 +1030,14 @@ int32_t moe_expert_rows(const void* xr, const int32_t* offsets, int32_t R, int32
   return MOE_OK;
 }
 
-int32_t moe_combine_rows(const void* y, const int32_t* row_of, int32_t T, int32_t H,
+int32_t moe_combine_rows(const void* y, int32_t R, const int32_t* row_of, int32_t T, int32_t H,
                          int32_t top_k, const void* shared, const void* residual, void* out,
                          void* stream) {
-  if (T < 0 || H <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (R < 0 || T < 0 || H <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
   if (H % 64 != 0 || H > MAX_DIM || top_k > MAX_TOPK) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) return MOE_OK;
   if (!y || !row_of || !out || out == y) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_combine_rows(y, row_of, top_k, T, H, shared, residual, out,
+  return cuda_status(launch_combine_rows(y, R, row_of, top_k, T, H, shared, residual, out,
                                          static_cast<cudaStream_t>(stream)));
 }
 

@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(32)
 // One warp per token (small batches: up to H/256 warps, each on every
 // parts-th 512-byte column block); 16-byte loads and stores.
 __global__ void __launch_bounds__(256)
-    combine_rows_kernel(const __nv_bfloat16* __restrict__ y, const int* __restrict__ row_of,
+    combine_rows_kernel(const __nv_bfloat16* __restrict__ y, int R, const int* __restrict__ row_of,
                         int top_k, int T, int H, int parts,
                         const __nv_bfloat16* __restrict__ shared,
                         const __nv_bfloat16* __restrict__ residual,
@@ -96,9 +96,10 @@ __global__ void __launch_bounds__(256)
           s[2 * i + 1] += bf16_hi(w[i]);
         }
       };
-      for (int j = 0; j < top_k; ++j) {  // a rejected id adds 0, as in the restore
+      for (int j = 0; j < top_k; ++j) {  // a rejected id (or a row outside y) adds 0
         const int r = rows[j];
-        add(r >= 0 ? reinterpret_cast<const uint4*>(y + (size_t)r * H)[c] : make_uint4(0, 0, 0, 0));
+        add(r >= 0 && r < R ? reinterpret_cast<const uint4*>(y + (size_t)r * H)[c]
+                            : make_uint4(0, 0, 0, 0));
       }
       if (shared) add(reinterpret_cast<const uint4*>(shared + (size_t)t * H)[c]);
       if (residual) add(reinterpret_cast<const uint4*>(residual + (size_t)t * H)[c]);
@@ -125,7 +126,7 @@ cudaError_t launch_tile_prefix(const int* offsets, int groups, int* tiles, cudaS
   return launch_chained(tile_prefix_kernel, dim3(1), dim3(32), 0, stream, offsets, groups, tiles);
 }
 
-cudaError_t launch_combine_rows(const void* y, const int* row_of, int top_k, int T, int H,
+cudaError_t launch_combine_rows(const void* y, int R, const int* row_of, int top_k, int T, int H,
                                 const void* shared, const void* residual, void* out,
                                 cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
@@ -138,7 +139,7 @@ cudaError_t launch_combine_rows(const void* y, const int* row_of, int top_k, int
   long long grid = ((long long)T * parts + 7) / 8;
   if (grid > cap) grid = cap;
   return launch_chained(combine_rows_kernel, dim3((unsigned)grid), dim3(256), 0, stream,
-                        static_cast<const __nv_bfloat16*>(y), row_of, top_k, T, H, parts,
+                        static_cast<const __nv_bfloat16*>(y), R, row_of, top_k, T, H, parts,
                         static_cast<const __nv_bfloat16*>(shared),
                         static_cast<const __nv_bfloat16*>(residual),
                         static_cast<__nv_bfloat16*>(out));

@@ -105,7 +105,7 @@ def lib() -> ctypes.CDLL:
         "moe_rows_expert_ids": (i32, [vp, i32, i32, vp, vp]),
         "moe_expert_rows_workspace_bytes": (sz, [i32, i32, i32, i32]),
         "moe_expert_rows": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
-        "moe_combine_rows": (i32, [vp, vp, i32, i32, i32, vp, vp, vp, vp]),
+        "moe_combine_rows": (i32, [vp, i32, vp, i32, i32, i32, vp, vp, vp, vp]),
         "moe_rmsnorm": (i32, [vp, vp, ctypes.c_float, i32, i32, vp, vp]),
         "moe_read_device_status": (i32, [vp, ctypes.POINTER(i32), vp]),
         "moe_selftest_wait_timeout": (i32, [vp, i64, vp]),
@@ -476,7 +476,8 @@ def combine_rows(y: torch.Tensor, row_of: torch.Tensor, top_k: int,
                  shared: Optional[torch.Tensor] = None, residual: Optional[torch.Tensor] = None,
                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """The restore through row_of (moe_combine_rows): out[t] = bf16(sum_j y[row_of[t, j]]
-    + shared[t] + residual[t]) in fp32, slot order, one rounding."""
+    + shared[t] + residual[t]) in fp32, slot order, one rounding; a row_of entry
+    outside [0, y.shape[0]) adds 0."""
     H = y.shape[1]
     T = row_of.numel() // top_k
     if y.dtype != torch.bfloat16 or y.dim() != 2 or not y.is_cuda or not y.is_contiguous():
@@ -489,7 +490,7 @@ def combine_rows(y: torch.Tensor, row_of: torch.Tensor, top_k: int,
         out = torch.empty((T, H), dtype=torch.bfloat16, device=y.device)
     else:
         _need(out, "out", torch.bfloat16, (T, H))
-    _check(lib().moe_combine_rows(_ptr(y), _ptr(row_of), T, H, top_k, _ptr(shared),
+    _check(lib().moe_combine_rows(_ptr(y), y.shape[0], _ptr(row_of), T, H, top_k, _ptr(shared),
                                   _ptr(residual), _ptr(out), _stream_ptr()), "moe_combine_rows")
     return out
 

@@ -241,11 +241,12 @@ def test_expert_parallel_entries_reject_bad_arguments_on_the_host(L):
     assert L.moe_expert_rows(*args(R=0, xr=None, y=None)) == 0
     # moe_combine_rows
     out = ctypes.c_void_p(0x30000)
-    assert L.moe_combine_rows(None, FAKE, 10, 256, 8, None, None, out, None) == 1
-    assert L.moe_combine_rows(FAKE, FAKE, 10, 256, 8, None, None, FAKE, None) == 1  # out is y
-    assert L.moe_combine_rows(FAKE, FAKE, 10, 250, 8, None, None, out, None) == 2
-    assert L.moe_combine_rows(FAKE, FAKE, 10, 256, 17, None, None, out, None) == 2
-    assert L.moe_combine_rows(None, None, 0, 256, 8, None, None, None, None) == 0
+    assert L.moe_combine_rows(None, 80, FAKE, 10, 256, 8, None, None, out, None) == 1
+    assert L.moe_combine_rows(FAKE, 80, FAKE, 10, 256, 8, None, None, FAKE, None) == 1  # out is y
+    assert L.moe_combine_rows(FAKE, -1, FAKE, 10, 256, 8, None, None, out, None) == 1  # R < 0
+    assert L.moe_combine_rows(FAKE, 80, FAKE, 10, 250, 8, None, None, out, None) == 2
+    assert L.moe_combine_rows(FAKE, 80, FAKE, 10, 256, 17, None, None, out, None) == 2
+    assert L.moe_combine_rows(None, 0, None, 0, 256, 8, None, None, None, None) == 0
 
 
 def test_public_header_is_plain_c():

@@ -46,3 +46,25 @@ def test_one_rank_ep_matches_oracle_and_the_block(T, H, E, I, k):
     # against the block: bit for bit
     diff = (out.float() - ref.float()).abs()
     assert torch.equal(out, ref), f"max diff {diff.max().item()}, {int((diff > 0).sum())} differ"
+
+
+def test_combine_rows_skips_rows_outside_y():
+    """moe_combine_rows: a row_of entry at or beyond y's row count, or negative,
+    adds 0 (like a rejected expert id); the rest is the fp32 sum in slot order."""
+    T, H, k, R = 50, 256, 4, 120
+    g = torch.Generator().manual_seed(7)
+    y = torch.randn((R, H), generator=g).to(torch.bfloat16)
+    row_of = torch.randint(0, R, (T, k), generator=g, dtype=torch.int32)
+    row_of[3, 1] = R           # one past the end
+    row_of[10, 0] = R + 1000   # far beyond
+    row_of[20, 2] = -1         # rejected
+    res = torch.randn((T, H), generator=g).to(torch.bfloat16)
+    out = ops.combine_rows(y.to(DEV), row_of.reshape(-1).to(DEV), k, residual=res.to(DEV))
+    torch.cuda.synchronize()
+    ref = torch.zeros((T, H), dtype=torch.float32)
+    for j in range(k):
+        r = row_of[:, j].long()
+        ok = (r >= 0) & (r < R)
+        ref[ok] += y[r[ok]].float()
+    ref += res.float()
+    assert torch.equal(out.cpu(), ref.to(torch.bfloat16))
