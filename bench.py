@@ -41,11 +41,11 @@ from routed_moe_layer_b200.ops import BlockConfig  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and TFLOP/s at T~19.4k bf16; % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-def kernels_per_step(T: int) -> int:
+def kernels_per_step(cfg: BlockConfig, fp8: bool = False) -> int:
     """Launches of one block forward: router 3 (Wr split, GEMM, selection), permutation
-    3 (one kernel up to 1024 tokens), gather, expert up, expert down (the shared expert
-    folded into both), combine."""
-    return 3 + (1 if T <= 1024 else 3) + 1 + 2 + 1
+    and gather (one kernel up to 1024 tokens, else three and a gather), expert up and
+    down (one launch for small batches; the shared expert folded into both), combine."""
+    return 3 + (1 if cfg.T <= 1024 else 4) + (1 if fused_small_batch(cfg, fp8) else 2) + 1
 
 
 def flops_per_token(cfg: BlockConfig) -> float:
@@ -70,12 +70,22 @@ def algorithmic_bytes(cfg: BlockConfig, experts_used: int, fp8: bool = False) ->
             cfg.E * 4 + 2.0 * cfg.T * cfg.H * 2)
 
 
-def up_launch_bytes(cfg: BlockConfig, experts_used: int, fp8: bool = False) -> float:
+def up_launch_bytes(cfg: BlockConfig, experts_used: int, fp8: bool = False,
+                    both: bool = False) -> float:
     """The expert-up launch's share of the algorithmic bytes: w13 of the used
-    experts, ws13 and the tokens x once (no intermediates)."""
+    experts, ws13 and the tokens x once (no intermediates); with ``both`` (one
+    launch runs both projections) also w2 of the used experts and ws2."""
     b = weight_bytes_per_element(fp8)
-    return (experts_used * 2.0 * cfg.I * cfg.H * b + 2.0 * cfg.I_shared * cfg.H * b +
+    k = 3.0 if both else 2.0
+    return (experts_used * k * cfg.I * cfg.H * b + k * cfg.I_shared * cfg.H * b +
             cfg.T * cfg.H * 2.0)
+
+
+def fused_small_batch(cfg: BlockConfig, fp8: bool) -> bool:
+    """The library runs both swapped projections as one launch: few rows per
+    expert and the shared expert, if any, a group of the routed GEMMs."""
+    return (not fp8 and cfg.T * cfg.top_k <= 64 * cfg.E and
+            (cfg.I_shared == cfg.I or cfg.I_shared == 0))
 
 
 class CallTimer:
@@ -464,6 +474,9 @@ def run_ours(args, world, rank, local):
         R = n_real * cfg.top_k
         up_rows = R + (wl.T if cfg.I_shared == cfg.I else 0)
         up_flops = 2.0 * up_rows * cfg.H * (2 * cfg.I)
+        both = not dense and fused_small_batch(cfg, fp8)
+        if both:  # the timed launch also runs the down projection
+            up_flops += 2.0 * up_rows * cfg.I * cfg.H
         if dense:  # the timed launch pair is the whole layer: both GEMMs
             up_rows, up_flops = wl.T, flops_per_step
         up_ms = up_ms_live
@@ -482,6 +495,8 @@ def run_ours(args, world, rank, local):
         kernel = ("grouped_gemm_swap_kernel<SwiGLU> (expert up, shared expert folded in)"
                   if swapped else
                   "grouped_gemm_kernel<SwiGLU> (expert up, shared expert folded in)")
+        if both:
+            kernel = "swap_fused_kernel (expert up then down in one launch, shared expert folded in)"
         if fp8:
             swapped = True  # FP8 weights: the dequantising swapped kernel at every size
             kernel = "grouped_gemm_swap_fp8_kernel<SwiGLU> (expert up, E4M3 weights, shared folded in)"
@@ -492,7 +507,7 @@ def run_ours(args, world, rank, local):
             # HBM-bound layer: the expert-up launch's algorithmic bytes are w13 of the
             # used experts, ws13 and the tokens once (the gathered rows it reads and
             # the h it writes are intermediates and are not counted)
-            up_bytes = up_launch_bytes(cfg, experts_used, fp8)
+            up_bytes = up_launch_bytes(cfg, experts_used, fp8, both)
             ach = up_bytes / (up_ms * 1e-3) / 1e9
             rf = {"bound": "hbm", "kernel": kernel, "achieved": ach, "peak": peaks["hbm_gbs"],
                   "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
@@ -544,7 +559,7 @@ def run_ours(args, world, rank, local):
                     "d2h_bytes_per_step": int(out_host.numel() * 2),
                     "mode": e2e_mode,
                     "serial_value": total_tokens / (e2e_serial_ms * 1e-3)},
-            "gpu_launches": ((2 if dense else kernels_per_step(wl.T) + (1 if layers > 1 else 0)) *
+            "gpu_launches": ((2 if dense else kernels_per_step(cfg, fp8) + (1 if layers > 1 else 0)) *
                              layers * args.steps),
             "clocks": sampler.summary(),
         }

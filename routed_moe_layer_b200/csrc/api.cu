@@ -49,7 +49,7 @@ int32_t check_cfg(const moe_cfg_t* c) {
 
 struct FwdLayout {
   size_t status, router, ids, w, blk_hist, offsets, mtiles, row_of, tok_of, w_of, pos_of, y, h,
-      hs, total;
+      hs, sched, y_sep, total;
 };
 
 // Slots per token of the token-major buffer of weighted expert outputs: the
@@ -69,6 +69,16 @@ bool use_swap(const moe_cfg_t& c) { return (int64_t)c.T * c.top_k <= 64LL * c.E;
 // Token rows per item of the swapped GEMMs: 32 when the experts average at
 // most 20 rows (so that few of them need a second chunk), else 128.
 int swap_chunk(const moe_cfg_t& c) { return (int64_t)c.T * c.top_k <= 20LL * c.E ? 32 : 128; }
+
+// Upper bound on the swapped GEMMs' chunks: every group adds at most one partial chunk.
+long long swap_chunk_bound(const moe_cfg_t& c) {
+  const long long R = (long long)c.T * c.top_k;
+  return R / swap_chunk(c) + c.E + (fuse_shared(c) ? 1 : 0) + 1;
+}
+
+// The swapped up and down projections run as one launch (grouped_gemm_swap_fused.cu)
+// when the shared expert, if any, is a group of them.
+bool fused_swap(const moe_cfg_t& c) { return use_swap(c) && (fuse_shared(c) || c.I_shared == 0); }
 
 FwdLayout fwd_layout(const moe_cfg_t& c) {
   FwdLayout L;
@@ -91,6 +101,12 @@ FwdLayout fwd_layout(const moe_cfg_t& c) {
   L.y = off;        off += align_up(std::max(R, T * (size_t)slots_per_token(c)) * c.H * 2);
   L.h = off;        off += align_up((R + (fuse_shared(c) ? T : 0)) * c.I * 2);
   L.hs = off;       off += align_up(fuse_shared(c) ? 0 : T * c.I_shared * 2);
+  // fused swapped projections: the item claim counter, then one ready counter per chunk;
+  // and a buffer of their own for the weighted outputs, which the down items write while
+  // other CTAs' up items may still read the gathered rows
+  L.sched = off;    off += align_up(fused_swap(c) ? (1 + swap_chunk_bound(c)) * 4 : 0);
+  L.y_sep = off;
+  off += align_up(fused_swap(c) ? T * (size_t)slots_per_token(c) * c.H * 2 : 0);
   L.total = off;
   return L;
 }
@@ -196,7 +212,7 @@ cudaError_t swap_gemms(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp, __n
                        __nv_bfloat16* hs, __nv_bfloat16* Y, const CUtensorMap& tm_w13,
                        const CUtensorMap& tm_w2, const CUtensorMap& tm_ws13,
                        const CUtensorMap& tm_ws2, const int* offsets, const PermuteOut& o,
-                       const GemmArgs& a, int sms, Rec& record, cudaStream_t s) {
+                       const GemmArgs& a, int* sched, int sms, Rec& record, cudaStream_t s) {
   const size_t T = c.T, R = T * c.top_k;
   const int slots = slots_per_token(c);
   const bool fused = fuse_shared(c);
@@ -217,51 +233,56 @@ cudaError_t swap_gemms(const moe_cfg_t& c, const void* x, __nv_bfloat16* xp, __n
     if ((e = make_tmap_2d_box(&tm_x, x, T, c.H, 32)) != cudaSuccess) return e;
     if (!fused && (e = make_tmap_2d_box(&tm_hs, hs, T, c.I_shared, 32)) != cudaSuccess) return e;
   }
-  if ((e = record(MOE_STAGE_EXPERT_UP)) != cudaSuccess) return e;
-  {  // h[r, i] = silu(W13g[i] . x_r) * (W13u[i] . x_r) per group (shared expert: group E)
-    GemmArgs g = a;
-    g.mtile_start = o.mtile_start;
-    g.row_start = offsets;
-    g.num_groups = groups;
-    if (fused) {  // shared rows: A from x at (row - group start)
-      g.alt_group = c.E;
-      g.alt_rebase = 1;
-    }
-    g.n_tiles = (c.I + 127) / 128;
-    g.k_steps = c.H / 64;
-    g.n_out_tile = 128;
-    g.b_second = c.I;
-    g.out = h;
-    g.ldo = c.I;
-    g.n_valid = c.I;
-    const int grid = (int)std::min<long long>(sms, chunk_bound * g.n_tiles);
-    if ((e = launch_grouped_gemm_swap(EPI_SWIGLU, chunk, tm_w13, tm_xp, tm_ws13, tm_x, g, grid,
-                                      s)) !=
-        cudaSuccess)
-      return e;
+  // h[r, i] = silu(W13g[i] . x_r) * (W13u[i] . x_r) per group (shared expert: group E)
+  GemmArgs gu = a;
+  gu.mtile_start = o.mtile_start;
+  gu.row_start = offsets;
+  gu.num_groups = groups;
+  if (fused) {  // shared rows: A from x at (row - group start)
+    gu.alt_group = c.E;
+    gu.alt_rebase = 1;
   }
-  if ((e = record(MOE_STAGE_EXPERT_DOWN)) != cudaSuccess) return e;
-  {  // Y[pos_r, n] = w_r * (W2[n] . h_r) per expert; shared rows to slot top_k, unscaled
-    GemmArgs g = a;
-    g.mtile_start = o.mtile_start;
-    g.row_start = offsets;
-    g.num_groups = groups;
-    if (fused) {  // shared rows: A from h at their own rows, weights ws2, unscaled
-      g.alt_group = c.E;
-      g.alt_rebase = 0;
-    }
-    g.n_tiles = (c.H + 127) / 128;
-    g.k_steps = c.I / 64;
-    g.n_out_tile = 128;
-    g.out = Y;
-    g.ldo = c.H;
-    g.n_valid = c.H;
-    g.row_scale = o.w_of;
-    g.dest_pos = o.pos_of;
-    g.dest_mul = slots;
-    g.dest_add = c.top_k;
-    const int grid = (int)std::min<long long>(sms, chunk_bound * g.n_tiles);
-    if ((e = launch_grouped_gemm_swap(EPI_ROWSCALE, chunk, tm_w2, tm_h, tm_ws2, tm_h, g, grid,
+  gu.n_tiles = (c.I + 127) / 128;
+  gu.k_steps = c.H / 64;
+  gu.n_out_tile = 128;
+  gu.b_second = c.I;
+  gu.out = h;
+  gu.ldo = c.I;
+  gu.n_valid = c.I;
+  // Y[pos_r, n] = w_r * (W2[n] . h_r) per expert; shared rows to slot top_k, unscaled
+  GemmArgs gd = a;
+  gd.mtile_start = o.mtile_start;
+  gd.row_start = offsets;
+  gd.num_groups = groups;
+  if (fused) {  // shared rows: A from h at their own rows, weights ws2, unscaled
+    gd.alt_group = c.E;
+    gd.alt_rebase = 0;
+  }
+  gd.n_tiles = (c.H + 127) / 128;
+  gd.k_steps = c.I / 64;
+  gd.n_out_tile = 128;
+  gd.out = Y;
+  gd.ldo = c.H;
+  gd.n_valid = c.H;
+  gd.row_scale = o.w_of;
+  gd.dest_pos = o.pos_of;
+  gd.dest_mul = slots;
+  gd.dest_add = c.top_k;
+  if ((e = record(MOE_STAGE_EXPERT_UP)) != cudaSuccess) return e;
+  if (sched) {  // both projections in one launch (the expert_down stage is then empty)
+    const CUtensorMap maps[7] = {tm_w13, tm_xp, tm_ws13, tm_x, tm_w2, tm_h, tm_ws2};
+    const int grid =
+        (int)std::min<long long>(sms, chunk_bound * (gu.n_tiles + (long long)gd.n_tiles));
+    if ((e = launch_swap_fused(chunk, maps, gu, gd, sched, grid, s)) != cudaSuccess) return e;
+    if ((e = record(MOE_STAGE_EXPERT_DOWN)) != cudaSuccess) return e;
+  } else {
+    const int grid_u = (int)std::min<long long>(sms, chunk_bound * gu.n_tiles);
+    if ((e = launch_grouped_gemm_swap(EPI_SWIGLU, chunk, tm_w13, tm_xp, tm_ws13, tm_x, gu,
+                                      grid_u, s)) != cudaSuccess)
+      return e;
+    if ((e = record(MOE_STAGE_EXPERT_DOWN)) != cudaSuccess) return e;
+    const int grid_d = (int)std::min<long long>(sms, chunk_bound * gd.n_tiles);
+    if ((e = launch_grouped_gemm_swap(EPI_ROWSCALE, chunk, tm_w2, tm_h, tm_ws2, tm_h, gd, grid_d,
                                       s)) != cudaSuccess)
       return e;
   }
@@ -324,7 +345,9 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
   int* mtiles = at<int>(workspace, L.mtiles);
   int* row_of = at<int>(workspace, L.row_of);
   __nv_bfloat16* xp = at<__nv_bfloat16>(workspace, L.y);  // gathered rows, then ...
-  __nv_bfloat16* Y = xp;  // ... token-major weighted outputs (after the up projection)
+  // ... token-major weighted outputs (once the up projection has read them; in the
+  // fused swapped launch both run at once, so the outputs get a buffer of their own)
+  __nv_bfloat16* Y = fused_swap(c) ? at<__nv_bfloat16>(workspace, L.y_sep) : xp;
   __nv_bfloat16* h = at<__nv_bfloat16>(workspace, L.h);
   __nv_bfloat16* hs = at<__nv_bfloat16>(workspace, L.hs);
 
@@ -358,6 +381,11 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
   RouterParams rp = router_params(c);
   rp.clear_status = clear_status ? 1 : 0;
   rp.mask = opts ? opts->token_mask : nullptr;
+  int* sched = fused_swap(c) ? at<int>(workspace, L.sched) : nullptr;
+  if (sched) {  // the fused swapped projections' counters start at zero
+    rp.zero = sched;
+    rp.zero_n = (int)(1 + swap_chunk_bound(c));
+  }
   RMOE_TRY(launch_router(x, Wr, bias, rp, ids, tw, at<void>(workspace, L.router), status, timeout,
                          s));
 
@@ -389,8 +417,8 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
   a.alt_group = -1;
 
   if (use_swap(c)) {
-    RMOE_TRY(swap_gemms(c, x, xp, h, hs, Y, tm_w13, tm_w2, tm_ws13, tm_ws2, offsets, o, a, sms,
-                        record, s));
+    RMOE_TRY(swap_gemms(c, x, xp, h, hs, Y, tm_w13, tm_w2, tm_ws13, tm_ws2, offsets, o, a, sched,
+                        sms, record, s));
   } else {
     RMOE_TRY(record(MOE_STAGE_EXPERT_UP));
     {  // h = silu(A . W13g^T) * (A . W13u^T) per group: A = gathered rows (experts), x (shared)

@@ -175,28 +175,46 @@ __device__ __forceinline__ RowIn epilogue_row_inputs(const GemmArgs& a, const Ti
 }
 
 // One epilogue thread owns accumulator row r_in_tile and half `half` of the
-// tile's columns (two warps per TMEM lane quarter).
-template <int EPI>
+// tile's columns (two warps per TMEM lane quarter).  It reads its whole half
+// row into registers (back-to-back TMEM loads, one wait), hands the
+// accumulator back to the MMA warp (release(): the leader's tempty barrier)
+// and only then computes and stores, so that the next tiles' MMAs do not wait
+// for this tile's stores.
+template <int EPI, typename Release>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tbase,
                                               const TileCoord& tc, int r_in_tile, int half,
-                                              const RowIn& in) {
+                                              const RowIn& in, Release&& release) {
   const bool valid = r_in_tile < tc.rows;
   const int row = tc.row0 + r_in_tile;
+  uint32_t v[128];
   if constexpr (EPI == EPI_SWIGLU) {
-    // accumulator columns [0,128) gate, [128,256) up; output columns nt*128 + [0,128)
-    const int col0 = tc.nt * (BN / 2);
-#pragma unroll 1
-    for (int c = half * 64; c < half * 64 + 64; c += 32) {
-      uint32_t g[32], u[32];
-      tmem_ld_32x32b_x32(tbase + c, g);
-      tmem_ld_32x32b_x32(tbase + BN / 2 + c, u);
-      tmem_ld_wait();
+    // accumulator columns [0,128) gate, [128,256) up; this half: gate and up of
+    // output columns nt*128 + half*64 + [0,64), in v[0..63] and v[64..127]
+    tmem_ld_32x32b_x32(tbase + half * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
+    tmem_ld_32x32b_x32(tbase + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+    tmem_ld_32x32b_x32(tbase + BN / 2 + half * 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
+    tmem_ld_32x32b_x32(tbase + BN / 2 + half * 64 + 32,
+                       *reinterpret_cast<uint32_t(*)[32]>(v + 96));
+  } else {
+    // this half: accumulator columns half*128 + [0,128)
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      tmem_ld_32x32b_x32(tbase + half * 128 + 32 * c,
+                         *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
+  }
+  tmem_ld_wait();
+  release();
+  if constexpr (EPI == EPI_SWIGLU) {
+    const int col0 = tc.nt * (BN / 2) + half * 64;
+#pragma unroll
+    for (int c = 0; c < 64; c += 32) {
       if (valid && col0 + c < a.n_valid) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-          const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+          const float h0 = silu_f(__uint_as_float(v[c + 2 * i])) * __uint_as_float(v[64 + c + 2 * i]);
+          const float h1 =
+              silu_f(__uint_as_float(v[c + 2 * i + 1])) * __uint_as_float(v[64 + c + 2 * i + 1]);
           pk[i] = pack_bf16x2(h0, h1);
         }
         // 64 bytes of the row as two full-sector stores
@@ -206,19 +224,17 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tbase,
       }
     }
   } else {  // EPI_ROWSCALE: weighted rows scattered to their token-major slot
-    const int col0 = tc.nt * BN;
+    const int col0 = tc.nt * BN + half * 128;
     const float w = in.w;
     const int drow = in.drow;
-#pragma unroll 1
-    for (int c = half * 128; c < half * 128 + 128; c += 32) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tbase + c, v);
-      tmem_ld_wait();
+#pragma unroll
+    for (int c = 0; c < 128; c += 32) {
       if (valid && col0 + c < a.n_valid) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(w * __uint_as_float(v[2 * i]), w * __uint_as_float(v[2 * i + 1]));
+          pk[i] = pack_bf16x2(w * __uint_as_float(v[c + 2 * i]),
+                              w * __uint_as_float(v[c + 2 * i + 1]));
         // 64 bytes of the row as two full-sector stores
         __nv_bfloat16* dst = a.out + (size_t)drow * a.ldo + col0 + c;
         st_global_v8(dst, pk);
@@ -535,18 +551,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       tc_fence_after_sync();
       const uint32_t tbase =
           tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(q * 32) << 16);
+      // hand the accumulator back to the leader's MMA thread
+      const uint32_t tempty_leader = acc == 0 ? tempty_leader0 : tempty_leader1;
+      auto release = [&]() {
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(tempty_leader);
+      };
       if (!sw) {
-        epilogue_tile<EPI>(args, tbase, tc, r_in_tile, half, in);
-      } else if constexpr (EPI == EPI_ROWSCALE) {
-        epilogue_swapped_rowscale(args, tbase, whole, rank, q, half, lane);
+        epilogue_tile<EPI>(args, tbase, tc, r_in_tile, half, in, release);
       } else {
-        if (!epilogue_swapped_swiglu(args, tbase, whole, rank, q, half, lane, st, wc, xuses0,
-                                     xuses1))
-          break;
+        if constexpr (EPI == EPI_ROWSCALE) {
+          epilogue_swapped_rowscale(args, tbase, whole, rank, q, half, lane);
+        } else {
+          if (!epilogue_swapped_swiglu(args, tbase, whole, rank, q, half, lane, st, wc, xuses0,
+                                       xuses1))
+            break;
+        }
+        release();
       }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(acc == 0 ? tempty_leader0 : tempty_leader1);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }

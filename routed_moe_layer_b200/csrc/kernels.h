@@ -50,6 +50,8 @@ struct RouterParams {
   float rsf;
   int clear_status;  // 1: the router's first kernel clears the status word
   const uint8_t* mask = nullptr;  // [T] or null: 0 = padding token (ids -1, weights 0)
+  int* zero = nullptr;  // [zero_n] ints the router's first kernel sets to 0 (counters of
+  int zero_n = 0;       //   later kernels of the same forward), or null
 };
 
 // Router on the tensor cores: scratch holds the 3-term bf16 split of Wr and the
@@ -156,6 +158,17 @@ cudaError_t launch_grouped_gemm_swap(int epi, int chunk, const CUtensorMap& tmW,
                                      const CUtensorMap& tmX, const CUtensorMap& tmW2,
                                      const CUtensorMap& tmX2, const GemmArgs& args, int grid,
                                      cudaStream_t stream);
+
+// Both swapped projections in one persistent launch (grouped_gemm_swap_fused.cu):
+// up items (args up: EPI_SWIGLU, out = h) then down items (args dn:
+// EPI_ROWSCALE, reading h), claimed in order from sched[0]; sched[1 + chunk]
+// counts the chunk's finished up-item epilogue warps.  sched (1 + chunks ints)
+// must be zero at launch.  maps: w13, xp rows, ws13, x (the shared group's
+// rows), w2, h rows, ws2 -- row maps with 32-row boxes, weight maps with
+// 128-row boxes.  The shared expert, when present, is group up.alt_group of
+// both (its up rows read from x, its down rows from h where they are).
+cudaError_t launch_swap_fused(int chunk, const CUtensorMap* maps, const GemmArgs& up,
+                              const GemmArgs& dn, int* sched, int grid, cudaStream_t stream);
 
 // FP8 expert weights (grouped_gemm_swap_fp8.cu): UE8M0 scale exponents, one
 // per 128 x 128 block, [groups][rows][cols] for the routed experts (s) and

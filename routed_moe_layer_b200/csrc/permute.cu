@@ -13,8 +13,13 @@
 //               also the token-major slot position of every row.
 //   4. gather:  xp[row] = x[tok_of[row]], walking tokens in order so that each
 //               token row is read once (skipped when x is not given).
-// Up to PERMUTE_SMALL_T tokens, steps 1-3 run in one CTA (one token per
-// thread), which saves two launches on small batches.
+// Up to PERMUTE_SMALL_T tokens, steps 1-4 run in one launch: every CTA of a
+// small grid computes steps 1-3 for all tokens in shared memory (one token
+// per thread; the same deterministic result in each CTA, so no CTA waits for
+// another), CTA 0 writes the offsets, and each CTA writes the rows of, and
+// gathers, its own share of the tokens.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -168,20 +173,26 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
-// T <= PERMUTE_SMALL_T: count, scan and scatter in one CTA of 1024 threads
-// (one token per thread); the same rows as the three-kernel path.
+// T <= PERMUTE_SMALL_T: count, scan and scatter with one token per thread
+// (1024 threads); the same rows as the three-kernel path.  Every CTA computes
+// the whole permutation; CTA 0 writes the offsets; CTA b writes the rows of
+// tokens [b*per, (b+1)*per) and, when x is given, gathers them into xp.
+constexpr int SMALL_PER_MAX = 64;  // tokens per CTA
 __global__ void __launch_bounds__(1024)
     permute_small_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T,
                          int E, int top_k, int extra_rows, int* __restrict__ expert_offsets,
                          int* __restrict__ mtile_start, int* __restrict__ row_of,
                          int* __restrict__ tok_of, float* __restrict__ w_of,
                          int* __restrict__ pos_of, int slot_stride,
-                         const uint8_t* __restrict__ tmask, int* status) {
+                         const uint8_t* __restrict__ tmask, int* status,
+                         const __nv_bfloat16* __restrict__ x, int H, int per,
+                         __nv_bfloat16* __restrict__ xp) {
   __shared__ uint32_t masks[32][MAXE];
   __shared__ int wbase[32][MAXE];
   __shared__ int tot[MAXE];
   __shared__ int excl_rows[MAXE + 1];
   __shared__ int excl_tiles[MAXE + 1];
+  __shared__ int rows_sm[SMALL_PER_MAX][MAX_TOPK_PERMUTE];
   pdl_launch_dependents();
   pdl_wait();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -201,7 +212,7 @@ __global__ void __launch_bounds__(1024)
       if (e >= 0 && e < E) {
         my_e[j] = e;
         atomicOr(&masks[warp][e], 1u << lane);
-      } else {
+      } else if (blockIdx.x == 0) {
         report_error(status, MOE_ERR_DEVICE_INDEX, 1);
       }
     }
@@ -218,23 +229,41 @@ __global__ void __launch_bounds__(1024)
   __syncthreads();
   if (tid < 32) scan_experts_warp(tot, E, excl_rows, excl_tiles);
   __syncthreads();
-  write_offsets(excl_rows, excl_tiles, E, extra_rows, expert_offsets, mtile_start);
-  if (t >= T) return;
-  const uint32_t lower = (1u << lane) - 1u;
+  if (blockIdx.x == 0) write_offsets(excl_rows, excl_tiles, E, extra_rows, expert_offsets, mtile_start);
+  const int t_lo = blockIdx.x * per, t_hi = min(T, t_lo + per);
+  if (t >= t_lo && t < t_hi) {
+    const uint32_t lower = (1u << lane) - 1u;
 #pragma unroll
-  for (int j = 0; j < MAX_TOPK_PERMUTE; ++j) {
-    if (j >= top_k) break;
-    const size_t tj = (size_t)t * top_k + j;
-    const int e = my_e[j];
-    if (e < 0) {
-      row_of[tj] = -1;
-      continue;
+    for (int j = 0; j < MAX_TOPK_PERMUTE; ++j) {
+      if (j >= top_k) break;
+      const size_t tj = (size_t)t * top_k + j;
+      const int e = my_e[j];
+      int row = -1;
+      if (e >= 0) {
+        row = excl_rows[e] + wbase[warp][e] + __popc(masks[warp][e] & lower);
+        tok_of[row] = t;
+        if (w_of) w_of[row] = my_w[j];
+        if (pos_of) pos_of[row] = t * slot_stride + j;
+      }
+      row_of[tj] = row;
+      rows_sm[t - t_lo][j] = row;
     }
-    const int row = excl_rows[e] + wbase[warp][e] + __popc(masks[warp][e] & lower);
-    row_of[tj] = row;
-    tok_of[row] = t;
-    if (w_of) w_of[row] = my_w[j];
-    if (pos_of) pos_of[row] = t * slot_stride + j;
+  }
+  if (!x || !xp) return;
+  __syncthreads();
+  // gather: this CTA's tokens, 32-byte pieces of a row, every piece to each of
+  // the token's rows (x read once)
+  const int pieces = H / 16;
+  const int n = (t_hi - t_lo) * pieces;
+  for (int c = tid; c < n; c += 1024) {
+    const int tl = c / pieces, pc = c - tl * pieces;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(t_lo + tl) * H + 16 * pc);
+    const uint4 a = src[0], b = src[1];
+    const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    for (int j = 0; j < top_k; ++j) {
+      const int r = rows_sm[tl][j];
+      if (r >= 0) st_global_v8(xp + (size_t)r * H + 16 * pc, v);
+    }
   }
 }
 
@@ -337,11 +366,22 @@ cudaError_t launch_permute(const int32_t* topk_ids, const float* topk_w, const v
                            int H, int E, int top_k, const PermuteOut& o, cudaStream_t stream) {
   cudaError_t err;
   if (T <= PERMUTE_SMALL_T) {
-    err = launch_chained(permute_small_kernel, dim3(1), dim3(1024), 0, stream, topk_ids, topk_w, T,
-                         E, top_k, o.extra_rows, o.expert_offsets, o.mtile_start, o.row_of,
-                         o.tok_of, o.w_of, o.pos_of, o.slot_stride, o.mask, o.status);
+    // with a gather: about 8 tokens per CTA (at most one CTA per SM); without: one CTA
+    const bool gather = x && o.xp;
+    int grid = gather ? std::min(num_sms(), (T + 7) / 8) : 1;
+    if (grid < 1) grid = 1;
+    int per = (T + grid - 1) / grid;
+    if (per > SMALL_PER_MAX) {
+      per = SMALL_PER_MAX;
+      grid = (T + per - 1) / per;
+    }
+    err = launch_chained(permute_small_kernel, dim3(grid), dim3(1024), 0, stream, topk_ids, topk_w,
+                         T, E, top_k, o.extra_rows, o.expert_offsets, o.mtile_start, o.row_of,
+                         o.tok_of, o.w_of, o.pos_of, o.slot_stride, o.mask, o.status,
+                         static_cast<const __nv_bfloat16*>(gather ? x : nullptr), H, per,
+                         static_cast<__nv_bfloat16*>(gather ? o.xp : nullptr));
     if (err != cudaSuccess) return err;
-    return launch_gather(x, T, H, top_k, o, stream);
+    return cudaGetLastError();
   }
   const int nblk = (T + PT - 1) / PT;
   err = launch_chained(permute_count_kernel, dim3(nblk), dim3(PT), 0, stream, topk_ids, T, E,

@@ -65,13 +65,15 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, uint6
 
 __global__ void __launch_bounds__(256)
     router_split_kernel(const float* __restrict__ Wr, size_t n, __nv_bfloat16* __restrict__ Wr3,
-                        int* status, int clear_status) {
+                        int* status, int clear_status, int* __restrict__ zero, int zero_n) {
   pdl_launch_dependents();
   pdl_wait();
   if (clear_status && blockIdx.x == 0 && threadIdx.x == 0) {  // first kernel of a forward
     status[0] = 0;
     status[1] = 0;
   }
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < zero_n; i += gridDim.x * blockDim.x)
+    zero[i] = 0;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x) {
     const float w = Wr[i];
@@ -567,7 +569,7 @@ cudaError_t launch_router(const void* x, const float* Wr, const float* bias, con
   const size_t n = (size_t)E * H;
   const int split_grid = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
   cudaError_t err = launch_chained(router_split_kernel, dim3(split_grid), dim3(256), 0, stream, Wr,
-                                   n, Wr3, status, p.clear_status);
+                                   n, Wr3, status, p.clear_status, p.zero, p.zero ? p.zero_n : 0);
   if (err != cudaSuccess) return err;
   const int S = router_splits(H);
   // split the expert columns when token tiles x K chunks leave most SMs idle
