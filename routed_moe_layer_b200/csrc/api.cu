@@ -159,42 +159,6 @@ RouterParams router_params(const moe_cfg_t& c) {
     if (e_ != cudaSuccess) return MOE_ERR_CUDA; \
   } while (0)
 
-// A group's last tile with at most this many rows runs with swapped operands
-// inside the pair kernel (TailMaps): it then costs about its rows rounded to
-// 16 instead of a full 256-row tile, with the same bits.
-constexpr int TAIL_MAX_ROWS = 192;
-
-// The maps of the swapped last tiles of one pair-kernel launch.
-// SwiGLU: A rows (a, a2) in 32-row boxes, weights (w, w2) in 64-row boxes.
-cudaError_t tail_maps_swiglu(TailMaps* t, const void* a, uint64_t a_rows, const void* a2,
-                             uint64_t a2_rows, uint64_t K, const void* w, uint64_t groups,
-                             uint64_t w_rows, const void* w2, uint64_t w2_rows) {
-  cudaError_t e;
-  if ((e = make_tmap_2d_box(&t->x, a, a_rows, K, 32)) != cudaSuccess) return e;
-  if ((e = make_tmap_2d_box(&t->x2, a2 ? a2 : a, a2 ? a2_rows : a_rows, K, 32)) != cudaSuccess)
-    return e;
-  if ((e = make_tmap_3d_box(&t->w, w, groups, w_rows, K, 64)) != cudaSuccess) return e;
-  if ((e = make_tmap_3d_box(&t->w2, w2 ? w2 : w, w2 ? 1 : groups, w2 ? w2_rows : w_rows, K, 64)) !=
-      cudaSuccess)
-    return e;
-  t->max_rows = TAIL_MAX_ROWS;
-  return cudaSuccess;
-}
-
-// Weighted down projection: A rows (a, a2) in 32-row boxes, the regular weight maps.
-cudaError_t tail_maps_rowscale(TailMaps* t, const void* a, uint64_t a_rows, const void* a2,
-                               uint64_t a2_rows, uint64_t K, const CUtensorMap& w,
-                               const CUtensorMap& w2) {
-  cudaError_t e;
-  if ((e = make_tmap_2d_box(&t->x, a, a_rows, K, 32)) != cudaSuccess) return e;
-  if ((e = make_tmap_2d_box(&t->x2, a2 ? a2 : a, a2 ? a2_rows : a_rows, K, 32)) != cudaSuccess)
-    return e;
-  t->w = w;
-  t->w2 = w2;
-  t->max_rows = TAIL_MAX_ROWS;
-  return cudaSuccess;
-}
-
 // Host checks of moe_forward (the configuration already checked).
 int32_t check_forward_args(const moe_cfg_t& c, const void* x, const float* Wr, const float* bias,
                            const void* w13, const void* w2, const void* ws13, const void* ws2,
@@ -438,11 +402,7 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
       g.ldo = c.I;
       g.n_valid = c.I;
       const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
-      TailMaps tails;
-      RMOE_TRY(tail_maps_swiglu(&tails, xp, R, fused ? x : nullptr, T, c.H, w13, c.E,
-                                2 * (uint64_t)c.I, fused ? ws13 : nullptr,
-                                2 * (uint64_t)c.I_shared));
-      RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_xp, tm_w13, tm_x, tm_ws13, g, grid, s, &tails));
+      RMOE_TRY(launch_grouped_gemm(EPI_SWIGLU, tm_xp, tm_w13, tm_x, tm_ws13, g, grid, s));
     }
     RMOE_TRY(record(MOE_STAGE_EXPERT_DOWN));
     {  // Y[t*slots + j] = w_tj * (h . W2^T) per expert; shared rows to slot top_k, unscaled
@@ -466,10 +426,7 @@ int32_t forward_impl(const void* x, const float* Wr, const float* bias, const vo
       g.dest_mul = slots;
       g.dest_add = c.top_k;
       const int grid = (int)std::min<long long>(sms, 2LL * mt_bound * g.n_tiles);
-      TailMaps tails;
-      RMOE_TRY(tail_maps_rowscale(&tails, h, h_rows, nullptr, 0, c.I, tm_w2,
-                                  fused ? tm_ws2 : tm_w2));
-      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, tm_h, tm_ws2, g, grid, s, &tails));
+      RMOE_TRY(launch_grouped_gemm(EPI_ROWSCALE, tm_h, tm_w2, tm_h, tm_ws2, g, grid, s));
     }
     RMOE_TRY(record(MOE_STAGE_SHARED_EXPERT));
     if (c.I_shared > 0 && !fused) {

@@ -32,7 +32,6 @@
 // accumulators).  Every wait is bounded (common.cuh): on a timeout the CTA
 // records MOE_ERR_DEVICE_TIMEOUT, drains its TMA loads and MMAs, frees TMEM
 // and returns.
-#include <algorithm>
 #include <mutex>
 
 #include <cudaTypedefs.h>
@@ -59,10 +58,6 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN);
 constexpr int EPI_WARPS = EPI_THREADS / 32;
 constexpr unsigned FULL = 0xffffffffu;
-// swapped last tiles
-constexpr int XBOX = 32;                    // token rows per TMA box
-constexpr int XBOX_BYTES = XBOX * BK * 2;
-constexpr int XCH = 16;                     // token columns per epilogue chunk
 
 struct __align__(8) SmemTail {
   uint64_t full[STAGES];
@@ -70,16 +65,10 @@ struct __align__(8) SmemTail {
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
-  // swapped SwiGLU tiles: up values handed from the warp reading TMEM lanes
-  // 64..127 to the one reading the matching gate lanes 0..63, per warp pair
-  // (p), column half (h) and buffer (b)
-  uint64_t xfull[2][2][2];
-  uint64_t xempty[2][2][2];
   uint32_t tmem_base;
   int abort_flag;
   int mt_start[MAX_GROUPS + 1];
   int row_start[MAX_GROUPS + 1];
-  float xbuf[2][2][2][XCH][32];  // [p][h][b][column][lane]
 };
 
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
@@ -99,15 +88,6 @@ struct TileCoord {
   int g, row0, rows, nt;
   int gstart;  // first row of the group (0 for a single group)
 };
-
-// A tile runs with swapped operands (weights on M, its rows on N) when it is
-// a group's partial last tile with at most tail_max_rows rows.
-__device__ __forceinline__ bool swapped_tile(const TileCoord& c, const GemmArgs& a) {
-  return c.rows <= a.tail_max_rows && c.rows < TILE_M;
-}
-
-// MMA N of a swapped tile: its rows rounded up to 16 (each CTA holds half).
-__device__ __forceinline__ int swapped_n(const TileCoord& c) { return (c.rows + 15) & ~15; }
 
 __device__ __forceinline__ TileCoord tile_coord(int tile, const GemmArgs& a, const int* mts,
                                                 const int* rs) {
@@ -244,114 +224,12 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tbase,
   }
 }
 
-// Epilogue of a swapped tile, EPI_ROWSCALE: TMEM lane l of CTA `rank` holds
-// output column nt*n_out_tile + 128*rank + l, TMEM column n the tile's row
-// row0 + n; the two column halves of the epilogue warps take alternate
-// 16-column chunks.  Same arithmetic as epilogue_tile.
-__device__ __forceinline__ void epilogue_swapped_rowscale(const GemmArgs& a, uint32_t tbase,
-                                                          const TileCoord& tc, uint32_t rank,
-                                                          int q, int half, int lane) {
-  const int n_sw = swapped_n(tc);
-  const int col = tc.nt * a.n_out_tile + BM * (int)rank + q * 32 + lane;
-  const bool col_ok = col < a.n_valid;
-  const bool unweighted = tc.g == a.alt_group || !a.dest_pos;
-#pragma unroll 1
-  for (int n0 = XCH * half; n0 < n_sw; n0 += 2 * XCH) {
-    uint32_t v[XCH];
-    tmem_ld_32x32b_x16(tbase + n0, v);
-    tmem_ld_wait();
-#pragma unroll
-    for (int j = 0; j < XCH; ++j) {
-      const int n = n0 + j;
-      if (n < tc.rows) {  // warp-uniform
-        const int row = tc.row0 + n;
-        float w;
-        int drow;
-        if (unweighted) {
-          w = 1.0f;
-          drow = (row - (tc.g == a.alt_group ? tc.gstart : 0)) * a.dest_mul + a.dest_add;
-        } else {
-          w = a.row_scale ? a.row_scale[row] : 1.0f;
-          drow = a.dest_pos[row];
-        }
-        if (col_ok)
-          a.out[(size_t)drow * a.ldo + col] = __float2bfloat16_rn(w * __uint_as_float(v[j]));
-      }
-    }
-  }
-}
-
-// Epilogue of a swapped tile, EPI_SWIGLU: in CTA `rank`, TMEM lanes 0..63 hold
-// the gate rows of h columns i = nt*n_out_tile + 64*rank + l and lanes 64..127
-// the up rows of the same i.  A warp may read only its own lane quarter, so
-// the warp on the up lanes (q = 2, 3) hands each 16-column chunk to the warp on
-// the matching gate lanes (q - 2) through a shared-memory buffer (two per warp
-// pair and column half, with bounded waits on xfull / xempty), and that warp
-// writes h.  uses0 / uses1 count the uses of buffer 0 / 1 so far (the same
-// sequence in both warps of a pair).  Returns false when a wait gave up.
-__device__ __forceinline__ bool epilogue_swapped_swiglu(const GemmArgs& a, uint32_t tbase,
-                                                        const TileCoord& tc, uint32_t rank,
-                                                        int q, int half, int lane, SmemTail& st,
-                                                        const WaitCtx& wc, uint32_t& uses0,
-                                                        uint32_t& uses1) {
-  const int n_sw = swapped_n(tc);
-  const int p = q & 1;
-  const bool up_warp = q >= 2;
-  const int col = tc.nt * a.n_out_tile + (BM / 2) * (int)rank + 32 * p + lane;
-  const bool col_ok = col < a.n_valid;
-  int k = 0;
-#pragma unroll 1
-  for (int n0 = XCH * half; n0 < n_sw; n0 += 2 * XCH, ++k) {
-    const int b = k & 1;
-    uint32_t v[XCH];
-    tmem_ld_32x32b_x16(tbase + n0, v);
-    tmem_ld_wait();
-    float(*buf)[32] = st.xbuf[p][half][b];
-    const uint32_t par = (b ? uses1 : uses0) & 1u;
-    if (up_warp) {
-      const bool ok = mbar_wait(&st.xempty[p][half][b], par ^ 1u, wc, 31);
-      if (!__all_sync(FULL, ok)) return false;
-#pragma unroll
-      for (int j = 0; j < XCH; ++j) buf[j][lane] = __uint_as_float(v[j]);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&st.xfull[p][half][b]);
-    } else {
-      const bool ok = mbar_wait(&st.xfull[p][half][b], par, wc, 32);
-      if (!__all_sync(FULL, ok)) return false;
-      float u[XCH];
-#pragma unroll
-      for (int j = 0; j < XCH; ++j) u[j] = buf[j][lane];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&st.xempty[p][half][b]);
-      if (col_ok) {
-#pragma unroll
-        for (int j = 0; j < XCH; ++j) {
-          const int n = n0 + j;
-          if (n < tc.rows) {
-            const float h = silu_f(__uint_as_float(v[j])) * u[j];
-            a.out[(size_t)(tc.row0 + n) * a.ldo + col] = __float2bfloat16_rn(h);
-          }
-        }
-      }
-    }
-    if (b)
-      ++uses1;
-    else
-      ++uses0;
-  }
-  return true;
-}
-
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmA2,
-                        const __grid_constant__ CUtensorMap tmB2,
-                        const __grid_constant__ CUtensorMap tmX,
-                        const __grid_constant__ CUtensorMap tmX2,
-                        const __grid_constant__ CUtensorMap tmW,
-                        const __grid_constant__ CUtensorMap tmW2, const GemmArgs args) {
+                        const __grid_constant__ CUtensorMap tmB2, const GemmArgs args) {
   pdl_launch_dependents();
   pdl_wait();
   extern __shared__ uint8_t smem_raw[];
@@ -379,12 +257,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&st.tempty[b], 2 * EPI_WARPS);    // leader: every epilogue warp of both CTAs
     }
     mbar_init(&st.drain, 1);
-    for (int p = 0; p < 2; ++p)
-      for (int h = 0; h < 2; ++h)
-        for (int b = 0; b < 2; ++b) {
-          mbar_init(&st.xfull[p][h][b], 1);   // the up-lane warp's lane 0
-          mbar_init(&st.xempty[p][h][b], 1);  // the gate-lane warp's lane 0
-        }
     st.abort_flag = 0;
     fence_mbar_init();
   }
@@ -394,14 +266,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (args.alt_group >= 0) {
       tma_prefetch_desc(&tmA2);
       tma_prefetch_desc(&tmB2);
-    }
-    if (args.tail_max_rows > 0) {
-      tma_prefetch_desc(&tmX);
-      tma_prefetch_desc(&tmW);
-      if (args.alt_group >= 0) {
-        tma_prefetch_desc(&tmX2);
-        tma_prefetch_desc(&tmW2);
-      }
     }
   }
   __syncthreads();
@@ -431,29 +295,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       for (int tile = cluster; ok && tile < total; tile += nclusters) {
         const TileCoord tc = tile_coord(tile, args, st.mt_start, st.row_start);
         const bool alt = tc.g == args.alt_group;
-        const int rebase = alt && args.alt_rebase ? tc.gstart : 0;
-        const int b_grp = alt ? 0 : tc.g;
-        const bool sw = swapped_tile(tc, args);
-        // regular tile: this CTA's 128 A rows at the stage's start, its half of
-        // the B tile after them.  A CTA whose half of the tile holds no rows of
-        // the group skips its A load (its accumulator rows are never stored);
-        // the leader arms the barrier for the bytes that will actually arrive.
+        // this CTA's 128 A rows at the stage's start, its half of the B tile
+        // after them.  A CTA whose half of the tile holds no rows of the
+        // group skips its A load (its accumulator rows are never stored); the
+        // leader arms the barrier for the bytes that will actually arrive.
         const CUtensorMap* ma = alt ? &tmA2 : &tmA;
         const CUtensorMap* mb = alt ? &tmB2 : &tmB;
-        const int a_row = tc.row0 + BM * (int)rank - rebase;
+        const int a_row = tc.row0 + BM * (int)rank - (alt && args.alt_rebase ? tc.gstart : 0);
+        const int b_grp = alt ? 0 : tc.g;
         const int b_row = tc.nt * args.n_out_tile + (int)rank * args.b_second;
         const bool load_a = tc.rows > BM * (int)rank;
-        // swapped tile: this CTA's 128 weight rows at the stage's start (SwiGLU:
-        // 64 gate rows, then the matching 64 up rows), its half of the tile's
-        // rows after them in 32-row boxes
-        const CUtensorMap* mx = alt ? &tmX2 : &tmX;
-        const CUtensorMap* mw = alt ? &tmW2 : &tmW;
-        const int hn = swapped_n(tc) >> 1;
-        const int nb = (hn + XBOX - 1) / XBOX;
-        const int x_row = tc.row0 + hn * (int)rank - rebase;
-        const int w_row = tc.nt * args.n_out_tile + (EPI == EPI_SWIGLU ? BM / 2 : BM) * (int)rank;
-        const uint32_t tx = sw ? 2 * (A_BYTES + nb * XBOX_BYTES)
-                               : 2 * B_BYTES + A_BYTES + (tc.rows > BM ? A_BYTES : 0);
+        const uint32_t tx = 2 * B_BYTES + A_BYTES + (tc.rows > BM ? A_BYTES : 0);
         for (int ks = 0; ks < args.k_steps; ++ks) {
           if (!mbar_wait(&st.empty[stage], phase ^ 1u, wc, 10)) {
             ok = false;
@@ -462,18 +314,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           uint8_t* sa = smem + (size_t)stage * STAGE_BYTES;
           const uint32_t full_leader = mapa_shared(smem_u32(&st.full[stage]), 0);
           if (leader) mbar_arrive_expect_tx(&st.full[stage], tx);
-          if (!sw) {
-            if (load_a) tma_load_2d_pair(sa, ma, full_leader, ks * BK, a_row);
-            tma_load_3d_pair(sa + A_BYTES, mb, full_leader, ks * BK, b_row, b_grp);
-          } else {
-            tma_load_3d_pair(sa, mw, full_leader, ks * BK, w_row, b_grp);
-            if constexpr (EPI == EPI_SWIGLU)
-              tma_load_3d_pair(sa + A_BYTES / 2, mw, full_leader, ks * BK, args.b_second + w_row,
-                               b_grp);
-            for (int b = 0; b < nb; ++b)
-              tma_load_2d_pair(sa + A_BYTES + b * XBOX_BYTES, mx, full_leader, ks * BK,
-                               x_row + b * XBOX);
-          }
+          if (load_a) tma_load_2d_pair(sa, ma, full_leader, ks * BK, a_row);
+          tma_load_3d_pair(sa + A_BYTES, mb, full_leader, ks * BK, b_row, b_grp);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -497,10 +339,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = cluster; ok && tile < total; tile += nclusters) {
-        // a swapped tile: M = 256 weight rows, N = its rows rounded up to 16
-        const TileCoord tc = tile_coord(tile, args, st.mt_start, st.row_start);
-        const uint32_t idesc =
-            swapped_tile(tc, args) ? idesc_bf16_f32(TILE_M, swapped_n(tc)) : IDESC;
         if (!mbar_wait(&st.tempty[acc], acc_phase ^ 1u, wc, 20)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -515,7 +353,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           const uint64_t db = sdesc_kmajor_sw128(sa + A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes along K per UMMA_K=16
-            umma_bf16_ss_pair(d_tmem, da + 2 * kk, db + 2 * kk, idesc, (ks | kk) != 0 ? 1u : 0u);
+            umma_bf16_ss_pair(d_tmem, da + 2 * kk, db + 2 * kk, IDESC, (ks | kk) != 0 ? 1u : 0u);
           umma_commit_pair_mask(&st.empty[stage], 0x3);  // free the stage in both CTAs
           if (++stage == STAGES) {
             stage = 0;
@@ -540,12 +378,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&st.tempty[1]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    uint32_t xuses0 = 0u, xuses1 = 0u;  // swapped SwiGLU tiles: uses of each exchange buffer
     for (int tile = cluster; tile < total; tile += nclusters) {
-      const TileCoord whole = tile_coord(tile, args, st.mt_start, st.row_start);
-      const bool sw = swapped_tile(whole, args);
-      const TileCoord tc = cta_part(whole, rank);
-      const RowIn in = sw ? RowIn{0.f, 0} : epilogue_row_inputs<EPI>(args, tc, r_in_tile);
+      const TileCoord tc = cta_part(tile_coord(tile, args, st.mt_start, st.row_start), rank);
+      const RowIn in = epilogue_row_inputs<EPI>(args, tc, r_in_tile);
       const bool ok = mbar_wait(&st.tfull[acc], acc_phase, wc, 30);
       if (!__all_sync(FULL, ok)) break;  // warp-uniform exit
       tc_fence_after_sync();
@@ -558,18 +393,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(tempty_leader);
       };
-      if (!sw) {
-        epilogue_tile<EPI>(args, tbase, tc, r_in_tile, half, in, release);
-      } else {
-        if constexpr (EPI == EPI_ROWSCALE) {
-          epilogue_swapped_rowscale(args, tbase, whole, rank, q, half, lane);
-        } else {
-          if (!epilogue_swapped_swiglu(args, tbase, whole, rank, q, half, lane, st, wc, xuses0,
-                                       xuses1))
-            break;
-        }
-        release();
-      }
+      epilogue_tile<EPI>(args, tbase, tc, r_in_tile, half, in, release);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -601,22 +425,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int EPI>
 cudaError_t launch_epi(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmA2,
-                       const CUtensorMap& tmB2, const GemmArgs& args_in, int grid,
-                       cudaStream_t stream, const TailMaps* tails) {
+                       const CUtensorMap& tmB2, const GemmArgs& args, int grid,
+                       cudaStream_t stream) {
   static std::atomic<int> smem_set[MAX_DEVICES];
   const cudaError_t attr =
       set_smem_limit_per_device(grouped_gemm_kernel<EPI>, (int)SMEM_BYTES, smem_set);
   if (attr != cudaSuccess) return attr;
   grid &= ~1;  // clusters of two CTAs
   if (grid < 2) grid = 2;
-  GemmArgs args = args_in;
-  args.tail_max_rows = tails ? std::min(tails->max_rows, TILE_M - 1) : 0;
-  if (tails)
-    return launch_chained(grouped_gemm_kernel<EPI>, dim3(grid), dim3(THREADS), SMEM_BYTES, stream,
-                          tmA, tmB, tmA2, tmB2, tails->x, tails->x2, tails->w, tails->w2, args);
-  // no swapped tiles: the extra maps are never read
   return launch_chained(grouped_gemm_kernel<EPI>, dim3(grid), dim3(THREADS), SMEM_BYTES, stream,
-                        tmA, tmB, tmA2, tmB2, tmA, tmA2, tmB, tmB2, args);
+                        tmA, tmB, tmA2, tmB2, args);
 }
 
 }  // namespace
@@ -662,18 +480,13 @@ cudaError_t make_tmap_3d_box(CUtensorMap* map, const void* base, uint64_t groups
 
 cudaError_t launch_grouped_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
                                 const CUtensorMap& tmA2, const CUtensorMap& tmB2,
-                                const GemmArgs& args, int grid, cudaStream_t stream,
-                                const TailMaps* tails) {
+                                const GemmArgs& args, int grid, cudaStream_t stream) {
   if (args.mtile_start && args.num_groups > MAX_GROUPS) return cudaErrorInvalidValue;
-  // swapped SwiGLU tiles pair gate row i with up row b_second + i in 64-row halves
-  if (tails && epi == EPI_SWIGLU && (args.n_out_tile != BN / 2)) return cudaErrorInvalidValue;
-  if (tails && epi == EPI_ROWSCALE && (args.n_out_tile != BN || args.b_second != BM))
-    return cudaErrorInvalidValue;
   switch (epi) {
     case EPI_SWIGLU:
-      return launch_epi<EPI_SWIGLU>(tmA, tmB, tmA2, tmB2, args, grid, stream, tails);
+      return launch_epi<EPI_SWIGLU>(tmA, tmB, tmA2, tmB2, args, grid, stream);
     case EPI_ROWSCALE:
-      return launch_epi<EPI_ROWSCALE>(tmA, tmB, tmA2, tmB2, args, grid, stream, tails);
+      return launch_epi<EPI_ROWSCALE>(tmA, tmB, tmA2, tmB2, args, grid, stream);
     default:
       return cudaErrorInvalidValue;
   }

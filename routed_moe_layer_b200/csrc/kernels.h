@@ -112,7 +112,6 @@ struct GemmArgs {
   int dest_mul, dest_add;  //   row * dest_mul + dest_add
   int* status;
   unsigned long long timeout_ns;
-  int tail_max_rows;       // set by launch_grouped_gemm from its TailMaps (0: no swapped tiles)
 };
 
 // A: 2D map over [rows, K] bf16, box 64 x 128, 128B swizzle.
@@ -127,26 +126,10 @@ cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, uint64_t groups, ui
 cudaError_t make_tmap_3d_box(CUtensorMap* map, const void* base, uint64_t groups,
                              uint64_t n_rows, uint64_t K, uint32_t box_rows);
 
-// A group's last tile, when it holds at most max_rows (< 256) rows, can run
-// with swapped operands inside the same pair kernel: the weight rows on the
-// MMA's M = 256 and the tile's rows on N (rounded up to 16), so that its cost
-// follows its rows instead of a full 256-row tile.  It gives the same bits as
-// the regular tile.  The maps it needs:
-//   x, x2  the A rows (and the alt group's) with 32-row boxes (make_tmap_2d_box);
-//   w, w2  EPI_SWIGLU: the weights (and the alt group's) with 64-row boxes, so
-//          that each CTA holds 64 gate and the matching 64 up rows;
-//          EPI_ROWSCALE: the regular weight maps (128-row boxes).
-struct TailMaps {
-  CUtensorMap x, x2, w, w2;
-  int max_rows;  // tiles with fewer rows than this + 1 run swapped (0: none)
-};
-
 // tmA2/tmB2 serve group args.alt_group (A rows re-based to 0, B group 0).
-// tails: null, or the maps of the swapped last tiles.
 cudaError_t launch_grouped_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
                                 const CUtensorMap& tmA2, const CUtensorMap& tmB2,
-                                const GemmArgs& args, int grid, cudaStream_t stream,
-                                const TailMaps* tails = nullptr);
+                                const GemmArgs& args, int grid, cudaStream_t stream);
 
 // Swapped operands for few rows per group (grouped_gemm_swap.cu): tmW is the
 // weights' 3D map (box 64 x 128 x 1), tmX the rows' 2D map with 32-row boxes;
