@@ -85,6 +85,38 @@ def test_router_batch_isolation(H, E, k, G, g):
     assert rep["near_ties"] <= max(2, T // 20)
 
 
+@pytest.mark.parametrize("T,H,k,G,g,norm,masked", [
+    (20000, 2048, 8, 4, 2, True, False),  # the block's shape
+    (4500, 1024, 8, 8, 3, True, True),    # groups of 16, padding tokens
+    (4500, 512, 6, 2, 1, False, False),   # groups of 64, no renormalisation
+    (4500, 256, 16, 4, 4, True, False),   # every group kept: no group step, top-16
+    (9000, 768, 1, 2, 2, True, True),     # top-1
+])
+def test_large_batch_router_matches_small_batch_router(T, H, k, G, g, norm, masked):
+    """Above 4096 tokens the selection runs 16 lanes per token, below it one
+    warp per token; a token's ids and weights are the same bits either way (128
+    experts in groups of 16, 32 or 64, with and without the group step, top-1
+    to top-16, with and without renormalisation and padding), and match the
+    oracle."""
+    n = 700
+    cfg = BlockConfig(T=T, H=H, E=128, top_k=k, n_group=G, topk_group=g,
+                      norm_topk_prob=norm, routed_scaling_factor=2.5 if norm else 0.3)
+    d = inputs.make_block_inputs(T, H, seed=H + k, E=128, I=64, I_shared=0, unit_scale=True)
+    dd = _dev(d)
+    mask = None
+    if masked:
+        gen = torch.Generator().manual_seed(H)
+        mask = (torch.rand(T, generator=gen) > 0.25).to(torch.uint8).to(DEV)
+    ids, w = ops.route(dd["x"], dd["Wr"], dd["bias"], cfg, token_mask=mask)
+    ids_s, w_s = ops.route(dd["x"][:n].contiguous(), dd["Wr"], dd["bias"], cfg.with_tokens(n),
+                           token_mask=None if mask is None else mask[:n].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(ids_s, ids[:n]) and torch.equal(w_s, w[:n])
+    rep = parity.check_routing(ids, w, *[parity.to_np(d[m]) for m in ("x", "Wr", "bias")], cfg,
+                               token_mask=None if mask is None else mask.cpu().numpy())
+    assert rep["near_ties"] <= max(2, T // 20)
+
+
 def test_router_bias_forces_selection_not_weights():
     T, H = 200, 512
     cfg = BlockConfig(T=T, H=H)
