@@ -17,16 +17,20 @@
 // is bit for bit that of the bf16 kernel on those weights.
 //
 // Pipeline, per 128-wide K step (one scale block):
-//   warp 0, one thread  TMA: the fp8 weight tile(s) [128 rows x 128 B] and the
-//                       token tiles of both 64-wide K halves, into a raw stage
-//   warps 6..13         per K half: dequantise the weight tile(s) into a bf16
+//   warp 0, one thread  TMA: the fp8 weight tile(s) [128 rows x 128 B] into a
+//                       raw stage
+//   warp 22, one thread TMA: the token tiles of both 64-wide K halves into a
+//                       token stage (a ring of its own, so that the weight
+//                       loads run as far ahead as the raw stages allow)
+//   warps 6..21         per K half: dequantise the weight tile(s) into a bf16
 //                       stage in the 128-byte-swizzled K-major layout of a TMA
 //                       load, fence the writes to the async proxy, signal
 //   warp 1, one thread  per K half: 4 UMMA_K=16 steps per weight tile
 //   warps 2..5          epilogue of item i while the MMAs of item i+1 run
-// A raw stage is free again once the converter warps have read it and the MMAs
-// of both halves (which read its token tiles) have completed.  Every wait is
-// bounded (common.cuh).
+// A raw stage is free again as soon as the converter warps have read it, a
+// token stage once the MMAs of both halves have completed: the weight ring,
+// which carries the HBM stream, takes most of the shared memory and is never
+// held by the MMAs.  Every wait is bounded (common.cuh).
 #include <mutex>
 
 #include <cudaTypedefs.h>
@@ -42,16 +46,18 @@ constexpr int WM = 128;            // weight rows per item (the MMA's M)
 constexpr int BK = 64;             // K per MMA stage (one 128-byte bf16 row)
 constexpr int KB8 = 128;           // K per raw stage = scale block width
 constexpr int XBOX = 32;           // token rows per TMA box
-constexpr int CONV_WARPS = 8;
+constexpr int CONV_WARPS = 16;  // one 8-row swizzle atom of every weight tile each
 constexpr int EPI_WARPS = 4;
-constexpr int THREADS = 64 + 32 * EPI_WARPS + 32 * CONV_WARPS;  // 448
+constexpr int TOK_WARP = 2 + EPI_WARPS + CONV_WARPS;  // 22
+constexpr int THREADS = 32 * (TOK_WARP + 1);            // 736
 constexpr int MAX_GROUPS = 129;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COLS = 256;
 constexpr int RAW_TILE = WM * KB8;   // fp8 weight tile: 16 KB
 constexpr int W_BYTES = WM * BK * 2; // bf16 weight tile of one K half: 16 KB
 constexpr int XBOX_BYTES = XBOX * BK * 2;
-constexpr int MAX_RAW = 8;
+constexpr int MAX_RAW = 12;
+constexpr int MAX_TOK = 4;
 constexpr int MMA_STAGES = 2;
 constexpr unsigned FULL = 0xffffffffu;
 
@@ -59,17 +65,22 @@ template <int EPI, int CHUNK>
 struct Shape8 {
   static constexpr int NW = EPI == EPI_SWIGLU ? 2 : 1;  // weight tiles per stage
   static constexpr int X_HALF = CHUNK * BK * 2;          // token tile of one K half
-  static constexpr int RAW_BYTES = NW * RAW_TILE + 2 * X_HALF;
+  static constexpr int RAW_BYTES = NW * RAW_TILE;        // fp8 weights of one K step
+  static constexpr int TOK_BYTES = 2 * X_HALF;           // tokens of one K step
   static constexpr int MMA_BYTES = NW * W_BYTES;
   static constexpr int RAW_STAGES =
-      EPI == EPI_SWIGLU ? (CHUNK == 32 ? 3 : 2) : (CHUNK == 32 ? 7 : 3);
-  static_assert(RAW_STAGES <= MAX_RAW, "raw stage count");
+      EPI == EPI_SWIGLU ? (CHUNK == 32 ? 4 : 3) : (CHUNK == 32 ? 10 : 7);
+  static constexpr int TOK_STAGES = CHUNK == 32 ? 3 : 2;
+  static_assert(RAW_STAGES <= MAX_RAW && TOK_STAGES <= MAX_TOK, "stage counts");
 };
 
-template <int CHUNK>
+template <int EPI, int CHUNK>
 struct __align__(8) Tail8 {
+  static constexpr int TOKS = EPI == EPI_ROWSCALE ? CHUNK : 1;  // per-row epilogue inputs
   uint64_t raw_full[MAX_RAW];
   uint64_t raw_empty[MAX_RAW];
+  uint64_t tok_full[MAX_TOK];
+  uint64_t tok_empty[MAX_TOK];
   uint64_t mma_full[MMA_STAGES];
   uint64_t mma_empty[MMA_STAGES];
   uint64_t tfull[2];
@@ -79,15 +90,15 @@ struct __align__(8) Tail8 {
   int abort_flag;
   int ch_start[MAX_GROUPS + 1];
   int row_start[MAX_GROUPS + 1];
-  float tok_w[EPI_WARPS][CHUNK];
-  int tok_d[EPI_WARPS][CHUNK];
+  float tok_w[EPI_WARPS][TOKS];
+  int tok_d[EPI_WARPS][TOKS];
 };
 
 template <int EPI, int CHUNK>
 constexpr size_t smem_bytes8() {
   using S = Shape8<EPI, CHUNK>;
-  return 1024 + (size_t)S::RAW_STAGES * S::RAW_BYTES + (size_t)MMA_STAGES * S::MMA_BYTES +
-         sizeof(Tail8<CHUNK>);
+  return 1024 + (size_t)S::RAW_STAGES * S::RAW_BYTES + (size_t)S::TOK_STAGES * S::TOK_BYTES +
+         (size_t)MMA_STAGES * S::MMA_BYTES + sizeof(Tail8<EPI, CHUNK>);
 }
 
 __device__ __forceinline__ void mbar_wait_drain8(uint64_t* bar, uint32_t parity,
@@ -199,9 +210,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* raw_base = smem;
-  uint8_t* mma_base = smem + (size_t)S::RAW_STAGES * S::RAW_BYTES;
-  Tail8<CHUNK>& st =
-      *reinterpret_cast<Tail8<CHUNK>*>(mma_base + (size_t)MMA_STAGES * S::MMA_BYTES);
+  uint8_t* tok_base = raw_base + (size_t)S::RAW_STAGES * S::RAW_BYTES;
+  uint8_t* mma_base = tok_base + (size_t)S::TOK_STAGES * S::TOK_BYTES;
+  Tail8<EPI, CHUNK>& st =
+      *reinterpret_cast<Tail8<EPI, CHUNK>*>(mma_base + (size_t)MMA_STAGES * S::MMA_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int groups = args.row_start ? args.num_groups : 1;
@@ -214,7 +226,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::RAW_STAGES; ++s) {
       mbar_init(&st.raw_full[s], 1);
-      mbar_init(&st.raw_empty[s], CONV_WARPS + 1);  // converter warps + the MMA commit
+      mbar_init(&st.raw_empty[s], CONV_WARPS);  // every converter warp has read it
+    }
+    for (int s = 0; s < S::TOK_STAGES; ++s) {
+      mbar_init(&st.tok_full[s], 1);
+      mbar_init(&st.tok_empty[s], 1);  // the MMA commit after both halves
     }
     for (int s = 0; s < MMA_STAGES; ++s) {
       mbar_init(&st.mma_full[s], CONV_WARPS);
@@ -281,36 +297,26 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ------------------------------------------------ TMA producer
       int rs = 0;
       uint32_t rph = 0;
-      uint32_t armed = 0, armed_parity = 0;
+      uint32_t armed = 0, armed_parity = 0;  // raw stages: armed at least once / last parity
       bool ok = true;
       for (int item = blockIdx.x; ok && item < total; item += gridDim.x) {
         const Item it =
             item_coord8<CHUNK>(item, args.n_tiles, groups, st.ch_start, st.row_start);
         const bool alt = it.g == args.alt_group;
         const CUtensorMap* mw = alt ? &tmW2 : &tmW;
-        const CUtensorMap* mx = alt ? &tmX2 : &tmX;
         const int w_grp = alt ? 0 : it.g;
         const int w_row = it.mt * args.n_out_tile;
-        const int x_row = it.row0 - (alt && args.alt_rebase ? it.gstart : 0);
-        const int nb = (it.rows + XBOX - 1) / XBOX;
-        const uint32_t tx = S::NW * RAW_TILE + 2 * nb * XBOX_BYTES;
         for (int ks = 0; ks < k128; ++ks) {
           if (!mbar_wait(&st.raw_empty[rs], rph ^ 1u, wc, 50)) {
             ok = false;
             break;
           }
           uint8_t* sr = raw_base + (size_t)rs * S::RAW_BYTES;
-          uint8_t* sx = sr + S::NW * RAW_TILE;
-          mbar_arrive_expect_tx(&st.raw_full[rs], tx);
+          mbar_arrive_expect_tx(&st.raw_full[rs], S::NW * RAW_TILE);
           tma_load_3d(sr, mw, &st.raw_full[rs], ks * KB8, w_row, w_grp);
           if constexpr (S::NW == 2)
             tma_load_3d(sr + RAW_TILE, mw, &st.raw_full[rs], ks * KB8, args.b_second + w_row,
                         w_grp);
-#pragma unroll
-          for (int a = 0; a < 2; ++a)
-            for (int b = 0; b < nb; ++b)
-              tma_load_2d(sx + a * S::X_HALF + b * XBOX_BYTES, mx, &st.raw_full[rs],
-                          ks * KB8 + a * BK, x_row + b * XBOX);
           armed |= 1u << rs;
           armed_parity = (armed_parity & ~(1u << rs)) | (rph << rs);
           if (++rs == S::RAW_STAGES) {
@@ -325,11 +331,52 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_wait_drain8(&st.raw_full[s], (armed_parity >> s) & 1u, args.timeout_ns);
       }
     }
+  } else if (warp == TOK_WARP) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer of the token tiles
+      int ts = 0;
+      uint32_t tph = 0;
+      uint32_t armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < total; item += gridDim.x) {
+        const Item it =
+            item_coord8<CHUNK>(item, args.n_tiles, groups, st.ch_start, st.row_start);
+        const bool alt = it.g == args.alt_group;
+        const CUtensorMap* mx = alt ? &tmX2 : &tmX;
+        const int x_row = it.row0 - (alt && args.alt_rebase ? it.gstart : 0);
+        const int nb = (it.rows + XBOX - 1) / XBOX;
+        const uint32_t tx = 2 * nb * XBOX_BYTES;
+        for (int ks = 0; ks < k128; ++ks) {
+          if (!mbar_wait(&st.tok_empty[ts], tph ^ 1u, wc, 57)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sx = tok_base + (size_t)ts * S::TOK_BYTES;
+          mbar_arrive_expect_tx(&st.tok_full[ts], tx);
+#pragma unroll
+          for (int a = 0; a < 2; ++a)
+            for (int b = 0; b < nb; ++b)
+              tma_load_2d(sx + a * S::X_HALF + b * XBOX_BYTES, mx, &st.tok_full[ts],
+                          ks * KB8 + a * BK, x_row + b * XBOX);
+          armed |= 1u << ts;
+          armed_parity = (armed_parity & ~(1u << ts)) | (tph << ts);
+          if (++ts == S::TOK_STAGES) {
+            ts = 0;
+            tph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < S::TOK_STAGES; ++s)
+          if ((armed >> s) & 1u)
+            mbar_wait_drain8(&st.tok_full[s], (armed_parity >> s) & 1u, args.timeout_ns);
+      }
+    }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      int rs = 0, ms = 0;
-      uint32_t rph = 0, mph = 0;
+      int ts = 0, ms = 0;
+      uint32_t tph = 0, mph = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
@@ -342,11 +389,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * ACC_COLS;
         for (int ks = 0; ok && ks < k128; ++ks) {
-          if (!mbar_wait(&st.raw_full[rs], rph, wc, 52)) {  // the token tiles
+          if (!mbar_wait(&st.tok_full[ts], tph, wc, 52)) {  // the token tiles
             ok = false;
             break;
           }
-          const uint32_t sx = smem_u32(raw_base + (size_t)rs * S::RAW_BYTES + S::NW * RAW_TILE);
+          const uint32_t sx = smem_u32(tok_base + (size_t)ts * S::TOK_BYTES);
 #pragma unroll 1
           for (int a = 0; a < 2; ++a) {
             if (!mbar_wait(&st.mma_full[ms], mph, wc, 53)) {
@@ -373,10 +420,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
           if (!ok) break;
-          umma_commit(&st.raw_empty[rs]);  // its token tiles are read
-          if (++rs == S::RAW_STAGES) {
-            rs = 0;
-            rph ^= 1u;
+          umma_commit(&st.tok_empty[ts]);  // its token tiles are read
+          if (++ts == S::TOK_STAGES) {
+            ts = 0;
+            tph ^= 1u;
           }
         }
         if (!ok) break;
@@ -466,13 +513,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (acc == 0) acc_phase ^= 1u;
     }
   } else {
-    // ------------------------------------------------ converter warps 6..13
+    // ------------------------------------------------ converter warps 6..21
     // Lane mapping inside one 8-row swizzle atom: lanes 8i..8i+7 take rows i and
     // i+4 (four 16-byte chunks each), so that the eight 16-byte accesses of
     // every quarter warp fall on eight different bank groups under the 128-byte
     // swizzle (chunk c of row r sits at chunk c ^ (r & 7)); the row i+4 lanes
     // store their two bf16 chunks in the opposite order for the same reason.
-    const int cw = warp - 2 - EPI_WARPS;  // 0..7
+    const int cw = warp - 2 - EPI_WARPS;  // 0..15: rows 8cw..8cw+7 of every weight tile
     const int u = lane & 7;
     const int rr = (lane >> 3) + 4 * (u >> 2);  // row inside the atom
     const int cl = u & 3;                       // 16-byte chunk inside a K half
@@ -489,16 +536,24 @@ __global__ void __launch_bounds__(THREADS, 1)
       // scale-block rows of the weight tiles (128-row aligned: N offsets are multiples of 128)
       const int srow0 = w_row / KB8;
       const int srow1 = (args.b_second + w_row) / KB8;
+      // block scales: each K step's loaded one step ahead
+      int s_next[S::NW];
+      s_next[0] = __ldg(sexp + (size_t)srow0 * sc.cols);
+      if constexpr (S::NW == 2) s_next[S::NW - 1] = __ldg(sexp + (size_t)srow1 * sc.cols);
       for (int ks = 0; ks < k128; ++ks) {
+        Scale2 mul[S::NW];
+#pragma unroll
+        for (int t = 0; t < S::NW; ++t) mul[t] = scale_multipliers(s_next[t]);
+        if (ks + 1 < k128) {
+          s_next[0] = __ldg(sexp + (size_t)srow0 * sc.cols + ks + 1);
+          if constexpr (S::NW == 2)
+            s_next[S::NW - 1] = __ldg(sexp + (size_t)srow1 * sc.cols + ks + 1);
+        }
         const bool got = mbar_wait(&st.raw_full[rs], rph, wc, 55);
         if (!__all_sync(FULL, got)) {
           ok = false;
           break;
         }
-        Scale2 mul[S::NW];
-        mul[0] = scale_multipliers(__ldg(sexp + (size_t)srow0 * sc.cols + ks));
-        if constexpr (S::NW == 2)
-          mul[S::NW - 1] = scale_multipliers(__ldg(sexp + (size_t)srow1 * sc.cols + ks));
         const uint8_t* sr = raw_base + (size_t)rs * S::RAW_BYTES;
 #pragma unroll 1
         for (int a = 0; a < 2; ++a) {
@@ -510,9 +565,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint8_t* sm = mma_base + (size_t)ms * S::MMA_BYTES;
 #pragma unroll
           for (int t = 0; t < S::NW; ++t) {
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-              const int r = 8 * (cw + 8 * p) + rr;  // atoms cw and cw + 8: rows 0..127
+            {
+              const int r = 8 * cw + rr;  // atom cw
               const int sw = r & 7;
               const int c = 4 * a + cl;               // fp8 chunk: K 16c..16c+15
               const uint4 v = *reinterpret_cast<const uint4*>(sr + t * RAW_TILE + r * 128 +
@@ -582,7 +636,7 @@ cudaError_t launch_swap8(const CUtensorMap& tmW, const CUtensorMap& tmX, const C
                          const CUtensorMap& tmX2, const GemmArgs& args, const Fp8Scales& sc,
                          int grid, cudaStream_t stream) {
   constexpr size_t smem = smem_bytes8<EPI, CHUNK>();
-  static_assert(smem <= 227 * 1024, "shared memory");
+  static_assert(smem <= 227 * 1024, "shared memory");  // 232,448 bytes per block
   static std::atomic<int> smem_set[MAX_DEVICES];
   const cudaError_t attr =
       set_smem_limit_per_device(grouped_gemm_swap_fp8_kernel<EPI, CHUNK>, (int)smem, smem_set);
