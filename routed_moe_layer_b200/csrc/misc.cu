@@ -54,8 +54,11 @@ __global__ void __launch_bounds__(256)
 // the expert outputs): the weighted slot rows of token t sit contiguously at
 // Y[t*slots .. t*slots + slots-1] (routed slots, then the shared expert), so
 // one warp per token streams them with 512-byte coalesced loads and sums them
-// in fp32 in slot order, then adds the residual, then rounds once.
-__global__ void __launch_bounds__(256)
+// in fp32 in slot order, then adds the residual, then rounds once.  NS: the
+// slot capacity of the instantiation (slots <= NS), which sizes the per-lane
+// load buffer and so the registers a thread holds.
+template <int NS>
+__global__ void __launch_bounds__(256, NS <= 9 ? 4 : 2)
     combine_slots_kernel(const __nv_bfloat16* __restrict__ Y, const int* __restrict__ row_of,
                          int top_k, int T, int H, int slots, int parts,
                          const __nv_bfloat16* __restrict__ residual,
@@ -78,12 +81,12 @@ __global__ void __launch_bounds__(256)
       float s[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) s[i] = 0.f;
-      uint4 y[17];
+      uint4 y[NS];
 #pragma unroll
-      for (int j = 0; j < 17; ++j)
+      for (int j = 0; j < NS; ++j)
         if (j < slots) y[j] = ((skip >> j) & 1u) ? make_uint4(0, 0, 0, 0) : src[(size_t)j * hv + c];
 #pragma unroll
-      for (int j = 0; j < 17; ++j) {
+      for (int j = 0; j < NS; ++j) {
         if (j < slots) {
           const uint32_t w[4] = {y[j].x, y[j].y, y[j].z, y[j].w};
 #pragma unroll
@@ -145,7 +148,9 @@ cudaError_t launch_combine_slots(const void* Y, const int* row_of, int top_k, in
   if (parts < 1) parts = 1;
   long long grid = ((long long)T * parts + 7) / 8;
   if (grid > cap) grid = cap;
-  return launch_chained(combine_slots_kernel, dim3((unsigned)grid), dim3(256), 0, stream,
+  auto kernel = slots <= 5 ? combine_slots_kernel<5>
+               : slots <= 9 ? combine_slots_kernel<9> : combine_slots_kernel<17>;
+  return launch_chained(kernel, dim3((unsigned)grid), dim3(256), 0, stream,
                         static_cast<const __nv_bfloat16*>(Y), row_of, top_k, T, H, slots, parts,
                         static_cast<const __nv_bfloat16*>(residual),
                         static_cast<__nv_bfloat16*>(out));
