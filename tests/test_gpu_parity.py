@@ -213,6 +213,8 @@ FORWARD_CASES = [
     (700, 320, 16, 128, 128, 4, 4, 2),      # H not a multiple of 256: down/combine N tail
     (1000, 1024, 128, 768, 768, 8, 4, 2),   # several tiles per expert, ragged tails
     (2048, 2048, 128, 768, 768, 8, 4, 2),
+    (300, 256, 64, 128, 128, 12, 4, 4),     # top-12 + shared: 13 slots per token
+    (200, 512, 32, 128, 0, 16, 2, 2),       # top-16, no shared expert: 16 slots per token
 ]
 
 
