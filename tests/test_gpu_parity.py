@@ -229,6 +229,25 @@ def test_forward_matches_oracle(T, H, E, I, Is, k, G, g):
     assert rep["rms_rel"] < 1e-2, rep  # bf16 storage of h and Y: a few 1e-3
 
 
+@pytest.mark.parametrize("T,H,E,I,Is,k,G,g", [
+    (40, 16384, 8, 128, 128, 2, 1, 1),      # H at the limit; swapped GEMMs (10 rows per expert)
+    (600, 16384, 8, 128, 128, 2, 1, 1),     # H at the limit; pair GEMMs (150 rows per expert)
+    (64, 256, 8, 16384, 16384, 2, 1, 1),    # I at the limit; swapped GEMMs
+    (400, 256, 8, 16384, 0, 2, 1, 1),       # I at the limit; pair GEMMs, no shared expert
+    (300, 512, 128, 128, 128, 16, 16, 2),   # 128 experts in 16 groups of 8, top-16
+])
+def test_forward_at_size_limits(T, H, E, I, Is, k, G, g):
+    """The largest H and I the library accepts (16384), and the most groups
+    and experts per token, against the oracle."""
+    cfg = BlockConfig(T=T, H=H, E=E, I=I, I_shared=Is, top_k=k, n_group=G, topk_group=g)
+    d = inputs.make_block_inputs(T, H, seed=5 + T, E=E, I=I, I_shared=Is, unit_scale=True)
+    out, ids, w = _run(_dev(d), cfg)
+    dn = parity.np_inputs(d)
+    parity.check_routing(ids, w, dn["x"], dn["Wr"], dn["bias"], cfg)
+    rep = parity.check_output(out, ids, dn, cfg)
+    assert rep["rms_rel"] < 1e-2, rep
+
+
 def test_forward_residual_and_no_shared_expert():
     T, H, E, I = 513, 512, 32, 128
     for Is in (0, 128):
