@@ -248,6 +248,42 @@ def test_forward_at_size_limits(T, H, E, I, Is, k, G, g):
     assert rep["rms_rel"] < 1e-2, rep
 
 
+@pytest.mark.parametrize("T,E,k,Is", [
+    (50, 1, 1, 128),    # one expert: out = 2.5 * SwiGLU(x) + shared(x); swapped GEMMs
+    (500, 1, 1, 128),   # the same on the pair GEMMs
+    (300, 4, 4, 0),     # every token to every expert (top-k = E), no shared expert
+])
+def test_forward_degenerate_routing(T, E, k, Is):
+    """Routing with no choice left (a single expert, or top-k = E) against the oracle."""
+    H, I = 256, 128
+    cfg = BlockConfig(T=T, H=H, E=E, I=I, I_shared=Is, top_k=k, n_group=1, topk_group=1)
+    d = inputs.make_block_inputs(T, H, seed=17 + T + E, E=E, I=I, I_shared=Is, unit_scale=True)
+    out, ids, w = _run(_dev(d), cfg)
+    assert torch.equal(torch.sort(ids, 1).values.cpu(),
+                       torch.arange(E, dtype=torch.int32).expand(T, E)[:, :k])
+    np.testing.assert_allclose(w.sum(1).cpu().numpy(), 2.5, rtol=1e-5)
+    dn = parity.np_inputs(d)
+    rep = parity.check_output(out, ids, dn, cfg)
+    assert rep["rms_rel"] < 1e-2, rep
+
+
+def test_identical_tokens_give_identical_rows():
+    """1000 copies of one token route to the same experts and fill whole and
+    partial tiles at every position: every output row has the same bits (each
+    row's arithmetic does not depend on where it sits), and the row matches the
+    oracle."""
+    T, H = 1000, 512
+    cfg = BlockConfig(T=T, H=H, I=256, I_shared=256)
+    d = inputs.make_block_inputs(T, H, seed=23, I=256, I_shared=256, unit_scale=True)
+    d["x"] = d["x"][:1].expand(T, H).contiguous()
+    out, ids, w = _run(_dev(d), cfg)
+    assert torch.equal(ids, ids[:1].expand(T, -1)) and torch.equal(w, w[:1].expand(T, -1))
+    assert torch.equal(out, out[:1].expand(T, H))
+    dn = parity.np_inputs({k: v[:1] if k == "x" else v for k, v in d.items()})
+    rep = parity.check_output(out[:1], ids[:1], dn, cfg.with_tokens(1))
+    assert rep["rms_rel"] < 1e-2, rep
+
+
 def test_forward_residual_and_no_shared_expert():
     T, H, E, I = 513, 512, 32, 128
     for Is in (0, 128):
